@@ -1,0 +1,156 @@
+"""CPU oracle for the Orthrus dual-view decode step.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``.  The product library never imports,
+links or calls it, and it shares no code with the CUDA path.
+
+The arithmetic lives in ``orthrus_oracle.c`` (plain C, double precision,
+OpenMP over output rows).  This module only compiles it with gcc and marshals
+numpy arrays through ctypes.  Each function follows the technical summary of
+"Orthrus: Memory-Efficient Parallel Token Generation via Dual-View Diffusion"
+(gist.science page), sections 2.2 (mask M_diff) and 2.3 (verification,
+consensus and commitment); see the C file's header for the readings taken
+where the pages are silent.
+
+Parity pins (tests/test_oracle_pins.py): K=1 reduction to causal decode, DIFF
+permutation invariance, AR view = K sequential decodes, explicit-mask brute
+force, a library SDPA cross-check, closed forms, planted consensus, hand cases
+and the lossless toy decode loop.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "orthrus_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+DIFF = 0
+AR = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, -O2, OpenMP)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_attn.restype = ctypes.c_int
+        lib.oracle_attn.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, i32p, f32p, f32p, f32p, ctypes.c_double,
+            ctypes.c_int, i32p, f64p, ctypes.c_int]
+        lib.oracle_consensus.restype = None
+        lib.oracle_consensus.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, f32p, i32p, i32p, i32p, i32p]
+        lib.oracle_kv_commit.restype = ctypes.c_int
+        lib.oracle_kv_commit.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def attention(view: int, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+              ctx_lens: np.ndarray, scale: float = 0.0, rows=None,
+              n_threads: int = 0) -> np.ndarray:
+    """fp64 masked softmax attention of the DIFF (M_diff) or AR (causal) view.
+
+    q [B,K,Hq,D], caches [B,Hkv,S_max,D] (values exact in float32), ctx_lens [B].
+    Returns float64 [B,K,Hq,D], or [len(rows), D] when ``rows`` lists (b,i,h).
+    """
+    B, K, Hq, D = q.shape
+    _, Hkv, S_max, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k_cache = np.ascontiguousarray(k_cache, dtype=np.float32)
+    v_cache = np.ascontiguousarray(v_cache, dtype=np.float32)
+    ctx = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+    if rows is None:
+        out = np.empty((B, K, Hq, D), dtype=np.float64)
+        rp, n_rows = None, 0
+    else:
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+        n_rows = rows.shape[0]
+        out = np.empty((n_rows, D), dtype=np.float64)
+        rp = _ptr(rows, ctypes.c_int32)
+    rc = _load().oracle_attn(
+        int(view), B, Hq, Hkv, D, S_max, K, _ptr(ctx, ctypes.c_int32),
+        _ptr(q, ctypes.c_float), _ptr(k_cache, ctypes.c_float),
+        _ptr(v_cache, ctypes.c_float), float(scale), n_rows, rp,
+        _ptr(out, ctypes.c_double), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_attn: bad argument or capacity violation")
+    return out
+
+
+def consensus(logits: np.ndarray, proposed: np.ndarray):
+    """Greedy consensus.  Returns (accepted_len [B], next_token [B], argmax [B,K])."""
+    B, K, V = logits.shape
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    proposed = np.ascontiguousarray(proposed, dtype=np.int32)
+    acc = np.empty(B, dtype=np.int32)
+    nxt = np.empty(B, dtype=np.int32)
+    am = np.empty((B, K), dtype=np.int32)
+    _load().oracle_consensus(B, K, V, _ptr(logits, ctypes.c_float),
+                             _ptr(proposed, ctypes.c_int32),
+                             _ptr(acc, ctypes.c_int32), _ptr(nxt, ctypes.c_int32),
+                             _ptr(am, ctypes.c_int32))
+    return acc, nxt, am
+
+
+def kv_commit(k_cache: np.ndarray, v_cache: np.ndarray, k_blk, v_blk,
+              ctx_lens: np.ndarray, accepted: np.ndarray, K: int,
+              advance: bool = True) -> None:
+    """In-place commit of one layer: copy block slots 0..n-1 (if given), advance ctx.
+
+    Caches [B,Hkv,S_max,D] and blocks [B,K,Hkv,D] of any fixed-size dtype; the
+    copy is byte-exact.  ctx_lens (int32) is updated in place when ``advance``.
+    """
+    B, Hkv, S_max, D = k_cache.shape
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert ctx_lens.dtype == np.int32 and ctx_lens.flags.c_contiguous
+    acc = np.ascontiguousarray(accepted, dtype=np.int32)
+    kb = vb = None
+    if k_blk is not None:
+        assert k_blk.shape == (B, K, Hkv, D) and k_blk.dtype == k_cache.dtype
+        k_blk = np.ascontiguousarray(k_blk)
+        v_blk = np.ascontiguousarray(v_blk)
+        kb, vb = k_blk.ctypes.data, v_blk.ctypes.data
+    rc = _load().oracle_kv_commit(
+        k_cache.ctypes.data, v_cache.ctypes.data, kb, vb,
+        _ptr(ctx_lens, ctypes.c_int32), _ptr(acc, ctypes.c_int32),
+        B, Hkv, D, S_max, K, k_cache.dtype.itemsize, 1 if advance else 0)
+    if rc != 0:
+        raise ValueError("oracle_kv_commit: bad argument or capacity violation")
