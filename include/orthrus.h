@@ -1,0 +1,202 @@
+/*
+ * orthrus.h — C ABI of liborthrus.so, the B200 (sm_100a) hot path of one Orthrus
+ * dual-view diffusion decoding step:
+ *
+ *   1. orthrus_attn(DIFF)   the diffusion view's attention over the shared KV cache
+ *   2. orthrus_attn(AR)     the frozen AR view's verification attention, same cache
+ *   3. orthrus_consensus    greedy left-to-right consensus on the AR logits
+ *   4. orthrus_kv_commit    keep the accepted prefix; rollback = length truncation
+ *
+ * Source of the method: "Orthrus: Memory-Efficient Parallel Token Generation via
+ * Dual-View Diffusion" (gist.science technical summary), section 2.1 (two
+ * attention paths over one shared KV cache), section 2.2 (block mask M_diff),
+ * section 2.3 (parallel projection, structural verification, consensus and
+ * commitment); Orthrus-Qwen3 (agentlenshq.com blog), "how Orthrus works"
+ * (K = 32 tokens per block, single-step denoising, verification pass).
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory, keeps no state between calls and never synchronises
+ *     the device; work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and the call returns at once.
+ *   - Return value: ORTHRUS_OK (0) or a negative ORTHRUS_ERR_* code for errors
+ *     found on the host (bad argument, unsupported shape, misalignment, too
+ *     small a workspace, launch failure).  Nothing is enqueued on error.
+ *   - Errors only the device can see (a ctx_lens value over capacity, an
+ *     accepted length out of range, a bounded wait that gave up) are OR-ed into
+ *     the caller's int32 `status` word (device pointer, may be NULL) as
+ *     ORTHRUS_STATUS_* bits; the affected work is skipped, never trapped.  Read
+ *     the word after synchronising the stream.
+ *   - Tensors are dense, row-major, with the layouts stated per argument.
+ *   - Block slot i of sequence b sits at absolute position ctx_lens[b] + i;
+ *     slot 0 is the anchor.
+ *
+ * Numerics: bf16 (or fp32) inputs, fp32 accumulation, fp32 attention output.
+ */
+#ifndef ORTHRUS_H
+#define ORTHRUS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define ORTHRUS_API __attribute__((visibility("default")))
+#else
+#define ORTHRUS_API
+#endif
+
+typedef enum {
+    ORTHRUS_DIFF = 0, /* diffusion view: mask M_diff (context + whole block)  */
+    ORTHRUS_AR = 1    /* AR verification view: causal within the block        */
+} orthrus_view;
+
+typedef enum {
+    ORTHRUS_BF16 = 0,
+    ORTHRUS_F32 = 1
+} orthrus_dtype;
+
+#define ORTHRUS_OK 0
+#define ORTHRUS_ERR_ARG (-1)          /* NULL pointer, non-positive size, bad enum */
+#define ORTHRUS_ERR_UNSUPPORTED (-2)  /* shape the kernels do not cover           */
+#define ORTHRUS_ERR_ALIGN (-3)        /* pointer not 16-byte aligned              */
+#define ORTHRUS_ERR_WORKSPACE (-4)    /* workspace missing or too small           */
+#define ORTHRUS_ERR_LAUNCH (-5)       /* CUDA launch / attribute call failed      */
+#define ORTHRUS_ERR_DEVICE (-6)       /* no usable sm_100 device / driver entry   */
+
+#define ORTHRUS_STATUS_CAPACITY 0x1   /* ctx_lens[b] < 0 or ctx_lens[b] + K > S_max */
+#define ORTHRUS_STATUS_ACCEPT 0x2     /* accepted_len[b] outside [0, K]             */
+#define ORTHRUS_STATUS_TIMEOUT 0x4    /* an on-chip pipeline wait gave up          */
+
+/* Largest supported sizes (checked on the host). */
+#define ORTHRUS_MAX_HEAD_DIM 256
+#define ORTHRUS_MAX_BLOCK 128          /* K */
+#define ORTHRUS_MAX_LAYERS 64          /* per orthrus_kv_commit call */
+
+/*
+ * orthrus_attn_workspace_size — bytes of scratch orthrus_attn needs for these
+ * sizes on the CURRENT device (the split-KV partials: one fp32 [G*K, D] tile
+ * plus G*K log-sum-exp values per (CTA, KV segment) boundary).  Independent of
+ * the context lengths.  Returns 0 for invalid sizes.
+ */
+ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K,
+                                   orthrus_dtype dtype);
+
+/*
+ * orthrus_attn — one view's attention for one layer.
+ *
+ * For every sequence b, query head h (KV head g = h / (Hq/Hkv)) and block slot
+ * i in [0, K):
+ *     out[b,i,h,:] = sum_j softmax_j(scale * <q[b,i,h,:], k_cache[b,g,j,:]>) v_cache[b,g,j,:]
+ * over the visible keys j:
+ *     DIFF (mask M_diff; section 2.2 rules 1-2): j in [0, ctx_lens[b] + K)
+ *          — the clean context before the anchor plus the whole block,
+ *          bidirectionally;
+ *     AR   (structural verification; section 2.3): j in [0, ctx_lens[b] + i]
+ *          — causal within the block.
+ *
+ *   view      ORTHRUS_DIFF or ORTHRUS_AR.
+ *   dtype     element type of q, k_cache, v_cache (bf16 or fp32).
+ *   q         [B, K, Hq, D]      this view's block queries.
+ *   k_cache   [B, Hkv, S_max, D] shared cache; rows [0, ctx_lens[b]) hold the
+ *             committed context, rows [ctx_lens[b], ctx_lens[b]+K) hold THIS
+ *             view's block keys (written by the caller before the call).
+ *             Rows at and beyond ctx_lens[b]+K are never read.
+ *   v_cache   [B, Hkv, S_max, D] same for values.
+ *   ctx_lens  [B] int32 committed lengths (device memory, read on the device).
+ *   scale     softmax scale; <= 0 selects 1/sqrt(D).
+ *   out       [B, K, Hq, D] fp32.
+ *   workspace device scratch of at least orthrus_attn_workspace_size() bytes,
+ *             16-byte aligned; contents need no initialisation and are
+ *             clobbered.  Calls that overlap on the device must not share it.
+ *   status    optional device int32 (see ORTHRUS_STATUS_*).  A sequence whose
+ *             ctx_lens[b] is negative or leaves no room for the block
+ *             (ctx_lens[b] + K > S_max) sets ORTHRUS_STATUS_CAPACITY and its
+ *             outputs are left unspecified.
+ *
+ * Supported: Hq % Hkv == 0; D % 32 == 0, D <= 256; K <= 128; G*K <= 128 for
+ * bf16 with D == 128 (tensor-core path); any other accepted shape runs the
+ * CUDA-core path.  All pointers 16-byte aligned.
+ */
+ORTHRUS_API int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q,
+                 const void *k_cache, const void *v_cache,
+                 const int32_t *ctx_lens, int B, int Hq, int Hkv, int D,
+                 int S_max, int K, float scale, float *out, void *workspace,
+                 size_t workspace_bytes, int32_t *status, void *stream);
+
+/*
+ * orthrus_consensus_workspace_size — scratch bytes for orthrus_consensus
+ * (one packed (value, index) candidate per vocabulary chunk per row).
+ */
+ORTHRUS_API size_t orthrus_consensus_workspace_size(int B, int K, int V);
+
+/*
+ * orthrus_consensus — greedy consensus (section 2.3 "consensus and
+ * commitment": strict left-to-right, a proposal is accepted only while it equals
+ * the AR greedy token; at the first mismatch the AR token takes its place).
+ *
+ *   logits       [B, K, V] fp32 AR-view logits; row i scores the token after
+ *                block slot i, i.e. the candidate proposed[b, i].
+ *   proposed     [B, K] int32 diffusion-view proposals p_1..p_K.
+ *   accepted_len [B] int32 out: a_b = number of leading i with
+ *                proposed[b,i] == r[b,i], in [0, K], where
+ *                r[b,i] = argmax_v logits[b,i,v] (lowest index wins ties; NaN
+ *                ranks above every number, the first NaN wins; +0 == -0).
+ *   next_token   [B] int32 out: r[b, min(a_b, K-1)] — the AR correction token
+ *                (or, when all K proposals match, the last one), which becomes
+ *                the next block's anchor.
+ *   argmax_out   optional [B, K] int32 out: r itself (may be NULL).
+ *   workspace    >= orthrus_consensus_workspace_size(B, K, V) bytes, 16-byte
+ *                aligned, clobbered.
+ */
+ORTHRUS_API int orthrus_consensus(const float *logits, const int32_t *proposed, int B,
+                      int K, int V, int32_t *accepted_len, int32_t *next_token,
+                      int32_t *argmax_out, void *workspace,
+                      size_t workspace_bytes, int32_t *status, void *stream);
+
+/*
+ * orthrus_kv_commit — commit the accepted prefix of the block for every layer
+ * and advance the committed length once (section 2.3: commit the synchronised
+ * prefix and truncate the cache; rollback is a length change, no data moves).
+ *
+ * For each sequence b: n_b = min(accepted_len[b] + 1, K) block slots are kept
+ * (the anchor plus the accepted proposals, whose AR-view K/V are exact).
+ *   - If k_blks is NULL the block already sits in cache rows
+ *     [ctx_lens[b], ctx_lens[b]+K) (the AR view wrote it there) and nothing
+ *     is copied.
+ *   - Otherwise, for each layer l, block slots 0..n_b-1 of
+ *     k_blks[l] / v_blks[l] ([B, K, Hkv, D], the caller's AR staging buffers)
+ *     are copied into cache rows [ctx_lens[b], ctx_lens[b]+n_b) of
+ *     k_caches[l] / v_caches[l] ([B, Hkv, S_max, D]).
+ * Then ctx_lens[b] += n_b (once, not per layer).  Rows past the new length
+ * are garbage that the next block overwrites.
+ *
+ *   num_layers   1..ORTHRUS_MAX_LAYERS; the four pointer arrays are HOST
+ *                arrays of num_layers device pointers (ignored when k_blks is
+ *                NULL; then k_caches/v_caches may be NULL too).
+ *   accepted_len [B] int32 from orthrus_consensus.  A value outside [0, K], or
+ *                a ctx_lens[b] that would leave no room (ctx + K > S_max), sets
+ *                the matching status bit and sequence b is left untouched.
+ */
+ORTHRUS_API int orthrus_kv_commit(int num_layers, void *const *k_caches,
+                      void *const *v_caches, const void *const *k_blks,
+                      const void *const *v_blks, int32_t *ctx_lens,
+                      const int32_t *accepted_len, int B, int Hkv, int D,
+                      int S_max, int K, orthrus_dtype dtype, int32_t *status,
+                      void *stream);
+
+/* Human-readable text for an ORTHRUS_* return code (static storage). */
+ORTHRUS_API const char *orthrus_error_string(int code);
+
+/* Library ABI version: (major << 16) | minor. */
+ORTHRUS_API int orthrus_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORTHRUS_H */

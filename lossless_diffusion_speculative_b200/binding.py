@@ -1,0 +1,165 @@
+"""Thin ctypes binding of liborthrus.so (argument marshalling only).
+
+Every function here has the name of the C entry point it wraps and does nothing
+but read shapes and device pointers off torch tensors and forward them; all
+arithmetic runs in the library's CUDA kernels.  There is no CPU fallback: if the
+library is missing or the device cannot run it, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+from .build import LIB
+
+DIFF, AR = 0, 1
+BF16, F32 = 0, 1
+
+ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_WORKSPACE, ERR_LAUNCH, ERR_DEVICE = -1, -2, -3, -4, -5, -6
+STATUS_CAPACITY, STATUS_ACCEPT, STATUS_TIMEOUT = 0x1, 0x2, 0x4
+
+EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn",
+            "orthrus_consensus_workspace_size", "orthrus_consensus",
+            "orthrus_kv_commit", "orthrus_error_string", "orthrus_version")
+
+
+class OrthrusError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (code {code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load liborthrus.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(
+                f"liborthrus.so not found at {LIB}; build it with "
+                "`python -m lossless_diffusion_speculative_b200.build`")
+        L = ctypes.CDLL(LIB)
+        vp, sz, i32, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+        L.orthrus_attn_workspace_size.restype = sz
+        L.orthrus_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.orthrus_attn.restype = i32
+        L.orthrus_attn.argtypes = [i32, i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                   f32, vp, vp, sz, vp, vp]
+        L.orthrus_consensus_workspace_size.restype = sz
+        L.orthrus_consensus_workspace_size.argtypes = [i32, i32, i32]
+        L.orthrus_consensus.restype = i32
+        L.orthrus_consensus.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]
+        L.orthrus_kv_commit.restype = i32
+        L.orthrus_kv_commit.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                        i32, vp, vp]
+        L.orthrus_error_string.restype = ctypes.c_char_p
+        L.orthrus_error_string.argtypes = [i32]
+        L.orthrus_version.restype = i32
+        L.orthrus_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise OrthrusError(fn, rc, lib().orthrus_error_string(rc).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("liborthrus takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("liborthrus takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def orthrus_version() -> int:
+    return int(lib().orthrus_version())
+
+
+def orthrus_attn_workspace_size(B: int, Hq: int, Hkv: int, D: int, K: int,
+                                dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib().orthrus_attn_workspace_size(B, Hq, Hkv, D, K, _dtype_code(dtype)))
+
+
+def orthrus_attn(view: int, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 ctx_lens: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                 status: Optional[torch.Tensor] = None, scale: float = 0.0,
+                 stream=None) -> None:
+    """q [B,K,Hq,D], caches [B,Hkv,S_max,D] (bf16 or fp32), ctx_lens [B] int32,
+    out [B,K,Hq,D] fp32, workspace uint8 of orthrus_attn_workspace_size bytes."""
+    B, K, Hq, D = q.shape
+    _, Hkv, S_max, _ = k_cache.shape
+    assert ctx_lens.dtype == torch.int32 and out.dtype == torch.float32
+    rc = lib().orthrus_attn(int(view), _dtype_code(q.dtype), _ptr(q), _ptr(k_cache),
+                            _ptr(v_cache), _ptr(ctx_lens), B, Hq, Hkv, D, S_max, K,
+                            float(scale), _ptr(out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _ptr(status),
+                            _stream(stream))
+    _check("orthrus_attn", rc)
+
+
+def orthrus_consensus_workspace_size(B: int, K: int, V: int) -> int:
+    return int(lib().orthrus_consensus_workspace_size(B, K, V))
+
+
+def orthrus_consensus(logits: torch.Tensor, proposed: torch.Tensor, accepted_len: torch.Tensor,
+                      next_token: torch.Tensor, workspace: torch.Tensor,
+                      argmax_out: Optional[torch.Tensor] = None,
+                      status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """logits [B,K,V] fp32, proposed [B,K] int32 -> accepted_len [B], next_token [B]."""
+    B, K, V = logits.shape
+    assert logits.dtype == torch.float32 and proposed.dtype == torch.int32
+    rc = lib().orthrus_consensus(_ptr(logits), _ptr(proposed), B, K, V, _ptr(accepted_len),
+                                 _ptr(next_token), _ptr(argmax_out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _ptr(status), _stream(stream))
+    _check("orthrus_consensus", rc)
+
+
+def orthrus_kv_commit(ctx_lens: torch.Tensor, accepted_len: torch.Tensor, *, K: int, Hkv: int,
+                      D: int, S_max: int, dtype: torch.dtype = torch.bfloat16,
+                      num_layers: int = 1,
+                      k_caches: Optional[Sequence[torch.Tensor]] = None,
+                      v_caches: Optional[Sequence[torch.Tensor]] = None,
+                      k_blks: Optional[Sequence[torch.Tensor]] = None,
+                      v_blks: Optional[Sequence[torch.Tensor]] = None,
+                      status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Commit min(a+1, K) block slots (copying from staging when k_blks is given)
+    and advance ctx_lens once."""
+    B = ctx_lens.shape[0]
+
+    def arr(ts):
+        if ts is None:
+            return None
+        a = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+        return ctypes.cast(a, ctypes.c_void_p), a
+
+    packs = [arr(x) for x in (k_caches, v_caches, k_blks, v_blks)]
+    if k_blks is not None:
+        num_layers = len(k_blks)
+    rc = lib().orthrus_kv_commit(num_layers, *[p[0] if p else None for p in packs],
+                                 _ptr(ctx_lens), _ptr(accepted_len), B, Hkv, D, S_max, K,
+                                 _dtype_code(dtype), _ptr(status), _stream(stream))
+    _check("orthrus_kv_commit", rc)

@@ -1,0 +1,232 @@
+// liborthrus C ABI: host-side argument checks, launch configuration and the
+// choice between the tensor-core and CUDA-core attention paths.  Declarations
+// and the contract of every entry point are in include/orthrus.h.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace orthrus;
+
+namespace {
+
+constexpr int kVersion = (1 << 16) | 0;
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// SM count of the current device (queried per call: cheap, and correct when
+// the caller switches devices).
+int current_sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
+
+// CTAs per attention launch and key granularity, per path.
+struct AttnPlan {
+    bool tc;
+    int grid;
+    int min_keys;
+    int slots;
+};
+
+bool attn_shape_ok(int B, int Hq, int Hkv, int D, int S_max, int K, orthrus_dtype dt)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || K <= 0) return false;
+    if (Hq % Hkv) return false;
+    if (dt != ORTHRUS_BF16 && dt != ORTHRUS_F32) return false;
+    return true;
+}
+
+bool attn_shape_supported(int Hq, int Hkv, int D, int K)
+{
+    return D % 32 == 0 && D <= ORTHRUS_MAX_HEAD_DIM && K <= ORTHRUS_MAX_BLOCK &&
+           (int64_t)(Hq / Hkv) * K <= 4096;
+}
+
+AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dt, int sms)
+{
+    AttnPlan pl;
+    const int rows = (Hq / Hkv) * K;
+    pl.tc = attn_tc_supported(dt, D, rows);
+    pl.grid = pl.tc ? sms : 2 * sms;
+    pl.min_keys = pl.tc ? 128 : 64;
+    pl.slots = pl.grid + B * Hkv;
+    return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orthrus_version(void) { return kVersion; }
+
+const char *orthrus_error_string(int code)
+{
+    switch (code) {
+    case ORTHRUS_OK: return "ok";
+    case ORTHRUS_ERR_ARG: return "invalid argument";
+    case ORTHRUS_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case ORTHRUS_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case ORTHRUS_ERR_WORKSPACE: return "workspace missing or too small";
+    case ORTHRUS_ERR_LAUNCH: return "CUDA launch failed";
+    case ORTHRUS_ERR_DEVICE: return "no usable CUDA device";
+    default: return "unknown error";
+    }
+}
+
+size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dtype)
+{
+    if (!attn_shape_ok(B, Hq, Hkv, D, 1, K, dtype) || !attn_shape_supported(Hq, Hkv, D, K))
+        return 0;
+    const int sms = current_sm_count();
+    if (sms <= 0) return 0;
+    const AttnPlan pl = plan_attn(B, Hq, Hkv, D, K, dtype, sms);
+    return attn_ws_bytes(pl.slots, (Hq / Hkv) * K, D);
+}
+
+int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const void *k_cache,
+                 const void *v_cache, const int32_t *ctx_lens, int B, int Hq, int Hkv, int D,
+                 int S_max, int K, float scale, float *out, void *workspace,
+                 size_t workspace_bytes, int32_t *status, void *stream)
+{
+    if (view != ORTHRUS_DIFF && view != ORTHRUS_AR) return ORTHRUS_ERR_ARG;
+    if (!q || !k_cache || !v_cache || !ctx_lens || !out) return ORTHRUS_ERR_ARG;
+    if (!attn_shape_ok(B, Hq, Hkv, D, S_max, K, dtype)) return ORTHRUS_ERR_ARG;
+    if (K > S_max) return ORTHRUS_ERR_ARG;
+    if (!(scale == scale) || isinf(scale)) return ORTHRUS_ERR_ARG;
+    if (!attn_shape_supported(Hq, Hkv, D, K)) return ORTHRUS_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (workspace && !aligned16(workspace)))
+        return ORTHRUS_ERR_ALIGN;
+    const int sms = current_sm_count();
+    if (sms <= 0) return ORTHRUS_ERR_DEVICE;
+    const AttnPlan pl = plan_attn(B, Hq, Hkv, D, K, dtype, sms);
+    const int rows = (Hq / Hkv) * K;
+    const size_t need = attn_ws_bytes(pl.slots, rows, D);
+    if (!workspace || workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+
+    AttnArgs a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.ctx_lens = ctx_lens;
+    a.out = out;
+    a.ws_o = static_cast<float *>(workspace);
+    size_t o_bytes = ((size_t)pl.slots * rows * D * sizeof(float) + 255) & ~(size_t)255;
+    a.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes);
+    a.status = status;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    a.K = K;
+    a.view = view;
+    a.dtype = dtype;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+    a.scale_log2 = sc * kLog2e;
+    a.min_keys = pl.min_keys;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = pl.tc ? launch_attn_tc(a, pl.grid, st) : launch_attn_simt(a, pl.grid, st);
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+static void consensus_split(int B, int K, int V, int sms, int *splits, int *chunk)
+{
+    const int rows = B * K;
+    int s = (4 * sms + rows - 1) / rows;         // about four CTAs per SM in total
+    const int max_s = (V + 2047) / 2048;         // at least 2048 logits per CTA
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    int c = (V + s - 1) / s;
+    c = (c + 3) & ~3;                            // whole float4 groups
+    s = (V + c - 1) / c;
+    *splits = s;
+    *chunk = c;
+}
+
+size_t orthrus_consensus_workspace_size(int B, int K, int V)
+{
+    if (B <= 0 || K <= 0 || V <= 0 || K > ORTHRUS_MAX_BLOCK) return 0;
+    const int sms = current_sm_count();
+    if (sms <= 0) return 0;
+    int s, c;
+    consensus_split(B, K, V, sms, &s, &c);
+    return (size_t)B * K * s * sizeof(unsigned long long);
+}
+
+int orthrus_consensus(const float *logits, const int32_t *proposed, int B, int K, int V,
+                      int32_t *accepted_len, int32_t *next_token, int32_t *argmax_out,
+                      void *workspace, size_t workspace_bytes, int32_t *status, void *stream)
+{
+    if (!logits || !proposed || !accepted_len || !next_token) return ORTHRUS_ERR_ARG;
+    if (B <= 0 || K <= 0 || V <= 0) return ORTHRUS_ERR_ARG;
+    if (K > ORTHRUS_MAX_BLOCK || (int64_t)B * K > 65535) return ORTHRUS_ERR_UNSUPPORTED;
+    if (!aligned16(logits) || (workspace && !aligned16(workspace))) return ORTHRUS_ERR_ALIGN;
+    const int sms = current_sm_count();
+    if (sms <= 0) return ORTHRUS_ERR_DEVICE;
+    ConsensusArgs a;
+    consensus_split(B, K, V, sms, &a.splits, &a.chunk);
+    const size_t need = (size_t)B * K * a.splits * sizeof(unsigned long long);
+    if (!workspace || workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+    a.logits = logits;
+    a.proposed = proposed;
+    a.accepted = accepted_len;
+    a.next_token = next_token;
+    a.argmax_out = argmax_out;
+    a.ws = static_cast<unsigned long long *>(workspace);
+    a.status = status;
+    a.B = B;
+    a.K = K;
+    a.V = V;
+    const cudaError_t e = launch_consensus(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+int orthrus_kv_commit(int num_layers, void *const *k_caches, void *const *v_caches,
+                      const void *const *k_blks, const void *const *v_blks, int32_t *ctx_lens,
+                      const int32_t *accepted_len, int B, int Hkv, int D, int S_max, int K,
+                      orthrus_dtype dtype, int32_t *status, void *stream)
+{
+    if (!ctx_lens || !accepted_len) return ORTHRUS_ERR_ARG;
+    if (num_layers <= 0 || B <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || K <= 0 || K > S_max)
+        return ORTHRUS_ERR_ARG;
+    if (dtype != ORTHRUS_BF16 && dtype != ORTHRUS_F32) return ORTHRUS_ERR_ARG;
+    if (num_layers > ORTHRUS_MAX_LAYERS || B > 65535) return ORTHRUS_ERR_UNSUPPORTED;
+    CommitArgs a;
+    memset(&a, 0, sizeof(a));
+    a.elem_bytes = dtype == ORTHRUS_BF16 ? 2 : 4;
+    a.copy = k_blks != nullptr;
+    if (a.copy) {
+        if (!v_blks || !k_caches || !v_caches) return ORTHRUS_ERR_ARG;
+        if ((D * a.elem_bytes) % 16) return ORTHRUS_ERR_UNSUPPORTED;
+        for (int l = 0; l < num_layers; ++l) {
+            if (!k_caches[l] || !v_caches[l] || !k_blks[l] || !v_blks[l]) return ORTHRUS_ERR_ARG;
+            if (!aligned16(k_caches[l]) || !aligned16(v_caches[l]) || !aligned16(k_blks[l]) ||
+                !aligned16(v_blks[l]))
+                return ORTHRUS_ERR_ALIGN;
+            a.k_caches[l] = k_caches[l];
+            a.v_caches[l] = v_caches[l];
+            a.k_blks[l] = k_blks[l];
+            a.v_blks[l] = v_blks[l];
+        }
+    }
+    a.ctx_lens = ctx_lens;
+    a.accepted = accepted_len;
+    a.status = status;
+    a.num_layers = num_layers;
+    a.B = B;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    a.K = K;
+    const cudaError_t e = launch_kv_commit(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/orthrus.h"
+
+namespace orthrus {
+
+// Everything one attention launch needs, passed by value to the kernels.
+struct AttnArgs {
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *ctx_lens;
+    float *out;
+    float *ws_o;         // [slots, rows, D] split partials (O normalised)
+    float *ws_lse;       // [slots, rows]    log2-sum-exp of each partial
+    int32_t *status;
+    int B, Hq, Hkv, D, S_max, K;
+    int view;            // orthrus_view
+    int dtype;           // orthrus_dtype
+    float scale_log2;    // softmax scale * log2(e)
+    int min_keys;        // smallest key range worth a CTA
+};
+
+// Workspace layout shared by the attention paths: `slots` partial tiles.
+inline size_t attn_ws_bytes(int slots, int rows, int D)
+{
+    size_t o = (size_t)slots * rows * D * sizeof(float);
+    o = (o + 255) & ~(size_t)255;
+    return o + (size_t)slots * rows * sizeof(float) + 256;
+}
+
+cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);
+cudaError_t launch_attn_combine(const AttnArgs &p, int grid_main, cudaStream_t st);
+
+// Tensor-core path (bf16, D == 128, G*K <= 128).  Returns cudaErrorNotSupported
+// when the device or shape does not qualify.
+bool attn_tc_supported(int dtype, int D, int rows);
+cudaError_t launch_attn_tc(const AttnArgs &p, int grid, cudaStream_t st);
+
+struct ConsensusArgs {
+    const float *logits;
+    const int32_t *proposed;
+    int32_t *accepted;
+    int32_t *next_token;
+    int32_t *argmax_out;
+    unsigned long long *ws;   // [B*K, splits] packed (value, index) keys
+    int32_t *status;
+    int B, K, V, splits, chunk;
+};
+cudaError_t launch_consensus(const ConsensusArgs &p, cudaStream_t st);
+
+struct CommitArgs {
+    void *k_caches[ORTHRUS_MAX_LAYERS];
+    void *v_caches[ORTHRUS_MAX_LAYERS];
+    const void *k_blks[ORTHRUS_MAX_LAYERS];
+    const void *v_blks[ORTHRUS_MAX_LAYERS];
+    int32_t *ctx_lens;
+    const int32_t *accepted;
+    int32_t *status;
+    int num_layers, B, Hkv, D, S_max, K, elem_bytes;
+    int copy;
+};
+cudaError_t launch_kv_commit(const CommitArgs &p, cudaStream_t st);
+
+}  // namespace orthrus

@@ -157,19 +157,22 @@ def context_cache(w: Workload, layer: int, poison: bool = True) -> Tuple[np.ndar
     """K and V caches [B,Hkv,S_max,D] with the committed context rows filled.
 
     Rows at and beyond ctx_b hold NaN when ``poison`` (nothing may read them
-    before the block is installed); otherwise zeros.
+    before the block is installed); otherwise zeros.  Sequence b's rows are
+    drawn in order b = 0..B-1 from one stream per tensor.
     """
     ctx = w.ctx_lens()
     S = w.S_max
-    fill = np.nan if poison else 0.0
-    kc = np.full((w.B, w.Hkv, S, w.D), fill, dtype=np.float32)
-    vc = np.full((w.B, w.Hkv, S, w.D), fill, dtype=np.float32)
-    cmax = int(ctx.max())
-    kk = _normal(w, layer, T_K_CTX, (w.B, w.Hkv, cmax, w.D))
-    vv = _normal(w, layer, T_V_CTX, (w.B, w.Hkv, cmax, w.D))
+    fill = np.float32(np.nan if poison else 0.0)
+    kc = np.empty((w.B, w.Hkv, S, w.D), dtype=np.float32)
+    vc = np.empty((w.B, w.Hkv, S, w.D), dtype=np.float32)
+    rk, rv = _rng(w, layer, T_K_CTX), _rng(w, layer, T_V_CTX)
     for b in range(w.B):
-        kc[b, :, :ctx[b]] = kk[b, :, :ctx[b]]
-        vc[b, :, :ctx[b]] = vv[b, :, :ctx[b]]
+        c = int(ctx[b])
+        for dst, rng in ((kc, rk), (vc, rv)):
+            x = rng.standard_normal(size=(w.Hkv, c, w.D), dtype=np.float32)
+            x *= np.float32(w.value_scale)
+            dst[b, :, :c] = round_to_bf16(x) if w.dtype == "bf16" else x
+            dst[b, :, c:] = fill
     return kc, vc
 
 

@@ -1,0 +1,165 @@
+"""GPU parity of orthrus_attn (both views) against the fp64 oracle.
+
+Tolerance (both paths): max |gpu - oracle| <= 2e-3 * RMS(oracle output).
+Small workloads are compared element by element in full; full-size workloads
+(run in the launch configuration the benchmark times) on sampled rows the
+oracle computes one by one, including every sequence's first and last block
+slot and the first and last query head.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lossless_diffusion_speculative_b200 import binding as ob
+from lossless_diffusion_speculative_b200 import workloads as wl
+from gpu_util import assert_attn_close, run_attn, sample_rows, tdtype, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=4)
+def _inputs(name, layer, view):
+    return wl.layer_inputs(wl.WORKLOADS[name], layer, view, poison=True)
+
+
+def _gpu(w, li, view, status=None):
+    dt = tdtype(w)
+    out = run_attn(view, to_dev(li.q, dt), to_dev(li.k_cache, dt), to_dev(li.v_cache, dt),
+                   torch.from_numpy(li.ctx_lens).cuda(), dt, status=status)
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("view", [ob.DIFF, ob.AR])
+@pytest.mark.parametrize("name", ["tiny_f32", "qwen3_1p7b_layer"])
+def test_attention_full_compare(name, view):
+    w = wl.WORKLOADS[name]
+    li = _inputs(name, 0, view)
+    got = _gpu(w, li, view)
+    ref = oracle.attention(view, li.q, li.k_cache, li.v_cache, li.ctx_lens)
+    assert_attn_close(got, ref, f"{name}/{view}")
+
+
+@pytest.mark.parametrize("view", [ob.DIFF, ob.AR])
+@pytest.mark.parametrize("name", ["qwen3_8b_step", "qwen3_4b_ragged", "qwen3_8b_long_k8",
+                                  "qwen3_8b_long_k16", "qwen3_8b_long_k32"])
+def test_attention_full_size_sampled(name, view):
+    w = wl.WORKLOADS[name]
+    li = _inputs(name, 0, view)
+    got = _gpu(w, li, view)
+    rows = sample_rows(w.B, w.K, w.Hq, 160, seed=view + 10 * w.cid)
+    ref = oracle.attention(view, li.q, li.k_cache, li.v_cache, li.ctx_lens, rows=rows)
+    assert_attn_close(got[rows[:, 0], rows[:, 1], rows[:, 2]], ref, f"{name}/{view}")
+
+
+def _custom(seed, B, Hq, Hkv, D, K, ctx, dtype="bf16", extra=0, scale=1 / np.sqrt(128)):
+    """Seeded edge-case inputs: rows past ctx+K poisoned with NaN."""
+    rng = np.random.default_rng(seed)
+    ctx = np.asarray(ctx, np.int32)
+    S = int(ctx.max()) + K + extra
+    S = (S + 7) // 8 * 8 if dtype == "bf16" else S
+    f = (lambda x: wl.round_to_bf16(x)) if dtype == "bf16" else (lambda x: x)
+    q = f(rng.standard_normal((B, K, Hq, D), dtype=np.float32) * np.float32(scale))
+    kc = np.full((B, Hkv, S, D), np.nan, np.float32)
+    vc = np.full((B, Hkv, S, D), np.nan, np.float32)
+    for b in range(B):
+        n = int(ctx[b]) + K
+        kc[b, :, :n] = f(rng.standard_normal((Hkv, n, D), dtype=np.float32) * np.float32(scale))
+        vc[b, :, :n] = f(rng.standard_normal((Hkv, n, D), dtype=np.float32) * np.float32(scale))
+    return q, kc, vc, ctx
+
+
+EDGE_CASES = {
+    # name: (B, Hq, Hkv, D, K, ctx list, dtype)
+    "block_only_C0": (1, 32, 8, 128, 32, [0], "bf16"),
+    "ragged_tile_edges": (9, 32, 8, 128, 32, [0, 1, 63, 64, 65, 127, 128, 129, 5003], "bf16"),
+    "K1_decode": (2, 32, 8, 128, 1, [777, 4096], "bf16"),
+    "K8": (2, 32, 8, 128, 8, [1000, 3], "bf16"),
+    "K16_G2": (3, 16, 8, 128, 16, [2222, 17, 640], "bf16"),
+    "K2_G1_mha": (2, 8, 8, 128, 2, [300, 1], "bf16"),
+    "G4_K20_odd": (2, 32, 8, 128, 20, [999, 1501], "bf16"),
+    "rows_over_128_simt": (1, 16, 2, 128, 32, [700], "bf16"),
+    "D64_bf16_simt": (2, 8, 2, 64, 8, [300, 45], "bf16"),
+    "D256_bf16_simt": (1, 4, 1, 256, 4, [129], "bf16"),
+    "f32_D128": (2, 8, 2, 128, 8, [200, 13], "f32"),
+}
+
+
+@pytest.mark.parametrize("view", [ob.DIFF, ob.AR])
+@pytest.mark.parametrize("case", list(EDGE_CASES))
+def test_attention_edge_cases(case, view):
+    B, Hq, Hkv, D, K, ctx, dt = EDGE_CASES[case]
+    q, kc, vc, ctx = _custom(100 + list(EDGE_CASES).index(case), B, Hq, Hkv, D, K, ctx, dt)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    got = run_attn(view, to_dev(q, tdt), to_dev(kc, tdt), to_dev(vc, tdt),
+                   torch.from_numpy(ctx).cuda(), tdt).cpu().numpy()
+    ref = oracle.attention(view, q, kc, vc, ctx)
+    assert_attn_close(got, ref, case)
+
+
+def test_exact_capacity_and_overflow_status():
+    """ctx + K == S_max is valid; a sequence with ctx + K > S_max sets the status
+    bit (no fault) and the other sequences are still exact."""
+    B, Hq, Hkv, D, K = 3, 32, 8, 128, 32
+    q, kc, vc, ctx = _custom(5, B, Hq, Hkv, D, K, [1000, 400, 64], extra=0)
+    S = kc.shape[2]
+    ctx_dev = ctx.copy()
+    ctx_dev[0] = S - K                      # exactly full
+    ctx_dev[2] = S - K + 1                  # one row over capacity
+    kc2, vc2 = kc.copy(), vc.copy()
+    rng = np.random.default_rng(6)
+    kc2[0, :, :S] = wl.round_to_bf16(rng.standard_normal((Hkv, S, D), dtype=np.float32) / 11.3)
+    vc2[0, :, :S] = wl.round_to_bf16(rng.standard_normal((Hkv, S, D), dtype=np.float32) / 11.3)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for view in (ob.DIFF, ob.AR):
+        got = run_attn(view, to_dev(q, torch.bfloat16), to_dev(kc2, torch.bfloat16),
+                       to_dev(vc2, torch.bfloat16), torch.from_numpy(ctx_dev).cuda(),
+                       torch.bfloat16, status=status).cpu().numpy()
+        ok = ctx_dev.copy()
+        ok[2] = 0
+        ref = oracle.attention(view, q[:2], kc2[:2], vc2[:2], ok[:2])
+        assert_attn_close(got[:2], ref, "capacity")
+    assert int(status.item()) & ob.STATUS_CAPACITY
+
+
+def test_negative_ctx_sets_status():
+    q, kc, vc, ctx = _custom(7, 2, 32, 8, 128, 8, [100, 50])
+    ctx[1] = -5
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = run_attn(ob.AR, to_dev(q, torch.bfloat16), to_dev(kc, torch.bfloat16),
+                   to_dev(vc, torch.bfloat16), torch.from_numpy(ctx).cuda(), torch.bfloat16,
+                   status=status).cpu().numpy()
+    assert int(status.item()) == ob.STATUS_CAPACITY
+    ref = oracle.attention(ob.AR, q[:1], kc[:1], vc[:1], ctx[:1])
+    assert_attn_close(got[:1], ref, "negative ctx")
+
+
+def test_custom_scale():
+    q, kc, vc, ctx = _custom(8, 1, 32, 8, 128, 32, [900])
+    got = run_attn(ob.DIFF, to_dev(q, torch.bfloat16), to_dev(kc, torch.bfloat16),
+                   to_dev(vc, torch.bfloat16), torch.from_numpy(ctx).cuda(), torch.bfloat16,
+                   scale=0.3).cpu().numpy()
+    assert_attn_close(got, oracle.attention(ob.DIFF, q, kc, vc, ctx, scale=0.3), "scale")
+
+
+def test_workspace_too_small_is_rejected():
+    q, kc, vc, ctx = _custom(9, 1, 32, 8, 128, 32, [100])
+    tq, tk, tv = (to_dev(x, torch.bfloat16) for x in (q, kc, vc))
+    out = torch.empty((1, 32, 32, 128), dtype=torch.float32, device="cuda")
+    need = ob.orthrus_attn_workspace_size(1, 32, 8, 128, 32, torch.bfloat16)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ob.OrthrusError) as ei:
+        ob.orthrus_attn(ob.DIFF, tq, tk, tv, torch.from_numpy(ctx).cuda(), out, ws)
+    assert ei.value.code == ob.ERR_WORKSPACE
+
+
+def test_repeatable_bitwise():
+    """Same inputs, same launch configuration -> bitwise identical output."""
+    q, kc, vc, ctx = _custom(10, 2, 32, 8, 128, 32, [3000, 700])
+    args = [to_dev(x, torch.bfloat16) for x in (q, kc, vc)]
+    c = torch.from_numpy(ctx).cuda()
+    a = run_attn(ob.AR, *args, c, torch.bfloat16)
+    b = run_attn(ob.AR, *args, c, torch.bfloat16)
+    assert torch.equal(a, b)
