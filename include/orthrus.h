@@ -189,6 +189,34 @@ ORTHRUS_API int orthrus_kv_commit(int num_layers, void *const *k_caches,
                       int S_max, int K, orthrus_dtype dtype, int32_t *status,
                       void *stream);
 
+/*
+ * orthrus_write_block — install a view's block K/V into the cache tail.
+ *
+ * The DIFF view's block (anchor + K-1 mask positions) and the AR view's block
+ * (anchor + the proposals) each occupy cache rows [ctx_lens[b], ctx_lens[b]+K)
+ * while that view's attention runs (section 2.1: both views work on one shared
+ * cache; section 2.3: the projected block is routed to the AR head).  For each
+ * layer l, all K slots of k_blks[l] / v_blks[l] ([B, K, Hkv, D]) are copied
+ * into rows [ctx_lens[b], ctx_lens[b]+K) of k_caches[l] / v_caches[l]
+ * ([B, Hkv, S_max, D]).  ctx_lens is only read.  A sequence with no room
+ * (ctx_lens[b] < 0 or ctx_lens[b] + K > S_max) sets ORTHRUS_STATUS_CAPACITY
+ * and is skipped.  The four pointer arrays are HOST arrays of num_layers
+ * device pointers (1..ORTHRUS_MAX_LAYERS); D * element size must be a
+ * multiple of 16 bytes.
+ */
+ORTHRUS_API int orthrus_write_block(int num_layers, void *const *k_caches,
+                                    void *const *v_caches, const void *const *k_blks,
+                                    const void *const *v_blks, const int32_t *ctx_lens,
+                                    int B, int Hkv, int D, int S_max, int K,
+                                    orthrus_dtype dtype, int32_t *status, void *stream);
+
+/*
+ * orthrus_attn_path — which attention kernel orthrus_attn runs for these sizes
+ * on the current device: 1 = tensor-core (tcgen05) path, 0 = CUDA-core path,
+ * or a negative ORTHRUS_ERR_* code.
+ */
+ORTHRUS_API int orthrus_attn_path(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dtype);
+
 /* Human-readable text for an ORTHRUS_* return code (static storage). */
 ORTHRUS_API const char *orthrus_error_string(int code);
 

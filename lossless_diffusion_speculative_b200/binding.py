@@ -21,9 +21,10 @@ BF16, F32 = 0, 1
 ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_WORKSPACE, ERR_LAUNCH, ERR_DEVICE = -1, -2, -3, -4, -5, -6
 STATUS_CAPACITY, STATUS_ACCEPT, STATUS_TIMEOUT = 0x1, 0x2, 0x4
 
-EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn",
+EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn", "orthrus_attn_path",
             "orthrus_consensus_workspace_size", "orthrus_consensus",
-            "orthrus_kv_commit", "orthrus_error_string", "orthrus_version")
+            "orthrus_kv_commit", "orthrus_write_block", "orthrus_error_string",
+            "orthrus_version")
 
 
 class OrthrusError(RuntimeError):
@@ -57,6 +58,11 @@ def lib():
         L.orthrus_kv_commit.restype = i32
         L.orthrus_kv_commit.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                         i32, vp, vp]
+        L.orthrus_write_block.restype = i32
+        L.orthrus_write_block.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                          i32, vp, vp]
+        L.orthrus_attn_path.restype = i32
+        L.orthrus_attn_path.argtypes = [i32, i32, i32, i32, i32, i32]
         L.orthrus_error_string.restype = ctypes.c_char_p
         L.orthrus_error_string.argtypes = [i32]
         L.orthrus_version.restype = i32
@@ -138,6 +144,34 @@ def orthrus_consensus(logits: torch.Tensor, proposed: torch.Tensor, accepted_len
     _check("orthrus_consensus", rc)
 
 
+def _ptr_array(ts):
+    """(void*, keep-alive) for a host array of device pointers, or (None, None)."""
+    if ts is None:
+        return None, None
+    a = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    return ctypes.cast(a, ctypes.c_void_p), a
+
+
+def orthrus_attn_path(B: int, Hq: int, Hkv: int, D: int, K: int,
+                      dtype: torch.dtype = torch.bfloat16) -> int:
+    """1 = tensor-core path, 0 = CUDA-core path (negative: error code)."""
+    return int(lib().orthrus_attn_path(B, Hq, Hkv, D, K, _dtype_code(dtype)))
+
+
+def orthrus_write_block(ctx_lens: torch.Tensor, k_caches: Sequence[torch.Tensor],
+                        v_caches: Sequence[torch.Tensor], k_blks: Sequence[torch.Tensor],
+                        v_blks: Sequence[torch.Tensor], status: Optional[torch.Tensor] = None,
+                        stream=None) -> None:
+    """Copy each layer's block K/V [B,K,Hkv,D] into cache rows [ctx, ctx+K)."""
+    B, Hkv, S_max, D = k_caches[0].shape
+    K = k_blks[0].shape[1]
+    packs = [_ptr_array(x) for x in (k_caches, v_caches, k_blks, v_blks)]
+    rc = lib().orthrus_write_block(len(k_caches), *[p[0] for p in packs], _ptr(ctx_lens), B, Hkv,
+                                   D, S_max, K, _dtype_code(k_caches[0].dtype), _ptr(status),
+                                   _stream(stream))
+    _check("orthrus_write_block", rc)
+
+
 def orthrus_kv_commit(ctx_lens: torch.Tensor, accepted_len: torch.Tensor, *, K: int, Hkv: int,
                       D: int, S_max: int, dtype: torch.dtype = torch.bfloat16,
                       num_layers: int = 1,
@@ -149,17 +183,10 @@ def orthrus_kv_commit(ctx_lens: torch.Tensor, accepted_len: torch.Tensor, *, K: 
     """Commit min(a+1, K) block slots (copying from staging when k_blks is given)
     and advance ctx_lens once."""
     B = ctx_lens.shape[0]
-
-    def arr(ts):
-        if ts is None:
-            return None
-        a = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
-        return ctypes.cast(a, ctypes.c_void_p), a
-
-    packs = [arr(x) for x in (k_caches, v_caches, k_blks, v_blks)]
+    packs = [_ptr_array(x) for x in (k_caches, v_caches, k_blks, v_blks)]
     if k_blks is not None:
         num_layers = len(k_blks)
-    rc = lib().orthrus_kv_commit(num_layers, *[p[0] if p else None for p in packs],
+    rc = lib().orthrus_kv_commit(num_layers, *[p[0] for p in packs],
                                  _ptr(ctx_lens), _ptr(accepted_len), B, Hkv, D, S_max, K,
                                  _dtype_code(dtype), _ptr(status), _stream(stream))
     _check("orthrus_kv_commit", rc)

@@ -48,14 +48,22 @@ bool attn_shape_supported(int Hq, int Hkv, int D, int K)
            (int64_t)(Hq / Hkv) * K <= 4096;
 }
 
+// `grid` is the number of split units: CTAs on the CUDA-core path, clusters on
+// the tensor-core path.
 AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dt, int sms)
 {
     AttnPlan pl;
     const int rows = (Hq / Hkv) * K;
-    pl.tc = attn_tc_supported(dt, D, rows);
-    pl.grid = pl.tc ? sms : 2 * sms;
-    pl.min_keys = pl.tc ? 128 : 64;
+    pl.tc = attn_tc_supported(dt, D, rows) && attn_tc_plan(&pl.grid, &pl.min_keys);
+    if (!pl.tc) {
+        pl.grid = 2 * sms;
+        pl.min_keys = 64;
+    }
     pl.slots = pl.grid + B * Hkv;
+    // equal-length segments split evenly when the unit count is a multiple of
+    // the segment count (no unit straddles a segment boundary)
+    const int segs = B * Hkv;
+    if (pl.grid >= segs) pl.grid -= pl.grid % segs;
     return pl;
 }
 
@@ -188,45 +196,89 @@ int orthrus_consensus(const float *logits, const int32_t *proposed, int B, int K
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 
-int orthrus_kv_commit(int num_layers, void *const *k_caches, void *const *v_caches,
-                      const void *const *k_blks, const void *const *v_blks, int32_t *ctx_lens,
-                      const int32_t *accepted_len, int B, int Hkv, int D, int S_max, int K,
-                      orthrus_dtype dtype, int32_t *status, void *stream)
+static int fill_layer_ptrs(CommitArgs &a, int num_layers, void *const *k_caches,
+                           void *const *v_caches, const void *const *k_blks,
+                           const void *const *v_blks, int D)
 {
-    if (!ctx_lens || !accepted_len) return ORTHRUS_ERR_ARG;
+    if (!k_blks || !v_blks || !k_caches || !v_caches) return ORTHRUS_ERR_ARG;
+    if ((D * a.elem_bytes) % 16) return ORTHRUS_ERR_UNSUPPORTED;
+    for (int l = 0; l < num_layers; ++l) {
+        if (!k_caches[l] || !v_caches[l] || !k_blks[l] || !v_blks[l]) return ORTHRUS_ERR_ARG;
+        if (!aligned16(k_caches[l]) || !aligned16(v_caches[l]) || !aligned16(k_blks[l]) ||
+            !aligned16(v_blks[l]))
+            return ORTHRUS_ERR_ALIGN;
+        a.k_caches[l] = k_caches[l];
+        a.v_caches[l] = v_caches[l];
+        a.k_blks[l] = k_blks[l];
+        a.v_blks[l] = v_blks[l];
+    }
+    a.copy = 1;
+    return ORTHRUS_OK;
+}
+
+static int commit_common(int num_layers, int B, int Hkv, int D, int S_max, int K,
+                         orthrus_dtype dtype, CommitArgs &a)
+{
     if (num_layers <= 0 || B <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || K <= 0 || K > S_max)
         return ORTHRUS_ERR_ARG;
     if (dtype != ORTHRUS_BF16 && dtype != ORTHRUS_F32) return ORTHRUS_ERR_ARG;
     if (num_layers > ORTHRUS_MAX_LAYERS || B > 65535) return ORTHRUS_ERR_UNSUPPORTED;
-    CommitArgs a;
     memset(&a, 0, sizeof(a));
     a.elem_bytes = dtype == ORTHRUS_BF16 ? 2 : 4;
-    a.copy = k_blks != nullptr;
-    if (a.copy) {
-        if (!v_blks || !k_caches || !v_caches) return ORTHRUS_ERR_ARG;
-        if ((D * a.elem_bytes) % 16) return ORTHRUS_ERR_UNSUPPORTED;
-        for (int l = 0; l < num_layers; ++l) {
-            if (!k_caches[l] || !v_caches[l] || !k_blks[l] || !v_blks[l]) return ORTHRUS_ERR_ARG;
-            if (!aligned16(k_caches[l]) || !aligned16(v_caches[l]) || !aligned16(k_blks[l]) ||
-                !aligned16(v_blks[l]))
-                return ORTHRUS_ERR_ALIGN;
-            a.k_caches[l] = k_caches[l];
-            a.v_caches[l] = v_caches[l];
-            a.k_blks[l] = k_blks[l];
-            a.v_blks[l] = v_blks[l];
-        }
-    }
-    a.ctx_lens = ctx_lens;
-    a.accepted = accepted_len;
-    a.status = status;
     a.num_layers = num_layers;
     a.B = B;
     a.Hkv = Hkv;
     a.D = D;
     a.S_max = S_max;
     a.K = K;
+    return ORTHRUS_OK;
+}
+
+int orthrus_kv_commit(int num_layers, void *const *k_caches, void *const *v_caches,
+                      const void *const *k_blks, const void *const *v_blks, int32_t *ctx_lens,
+                      const int32_t *accepted_len, int B, int Hkv, int D, int S_max, int K,
+                      orthrus_dtype dtype, int32_t *status, void *stream)
+{
+    if (!ctx_lens || !accepted_len) return ORTHRUS_ERR_ARG;
+    CommitArgs a;
+    int rc = commit_common(num_layers, B, Hkv, D, S_max, K, dtype, a);
+    if (rc != ORTHRUS_OK) return rc;
+    if (k_blks) {
+        rc = fill_layer_ptrs(a, num_layers, k_caches, v_caches, k_blks, v_blks, D);
+        if (rc != ORTHRUS_OK) return rc;
+    }
+    a.ctx_lens = ctx_lens;
+    a.accepted = accepted_len;
+    a.status = status;
     const cudaError_t e = launch_kv_commit(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+int orthrus_write_block(int num_layers, void *const *k_caches, void *const *v_caches,
+                        const void *const *k_blks, const void *const *v_blks,
+                        const int32_t *ctx_lens, int B, int Hkv, int D, int S_max, int K,
+                        orthrus_dtype dtype, int32_t *status, void *stream)
+{
+    if (!ctx_lens) return ORTHRUS_ERR_ARG;
+    CommitArgs a;
+    int rc = commit_common(num_layers, B, Hkv, D, S_max, K, dtype, a);
+    if (rc != ORTHRUS_OK) return rc;
+    rc = fill_layer_ptrs(a, num_layers, k_caches, v_caches, k_blks, v_blks, D);
+    if (rc != ORTHRUS_OK) return rc;
+    a.all_rows = 1;
+    a.ctx_lens = const_cast<int32_t *>(ctx_lens);      // read only in this mode
+    a.status = status;
+    const cudaError_t e = launch_kv_commit(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+int orthrus_attn_path(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dtype)
+{
+    if (!attn_shape_ok(B, Hq, Hkv, D, 1, K, dtype)) return ORTHRUS_ERR_ARG;
+    if (!attn_shape_supported(Hq, Hkv, D, K)) return ORTHRUS_ERR_UNSUPPORTED;
+    const int sms = current_sm_count();
+    if (sms <= 0) return ORTHRUS_ERR_DEVICE;
+    return plan_attn(B, Hq, Hkv, D, K, dtype, sms).tc ? 1 : 0;
 }
 
 }  // extern "C"

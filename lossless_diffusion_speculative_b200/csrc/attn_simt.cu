@@ -88,13 +88,21 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs p)
 }
 
 // Combine: for every segment covered by more than one CTA, merge the partials
-// with weights 2^(lse_s - max lse).  One warp per output row; lanes over D.
-__global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs p, int grid_main)
+// with weights 2^(lse_s - max lse) / sum.  One warp per output row; each lane
+// owns float4 columns, so every split contributes one coalesced row read per
+// warp.  The split weights are computed once per row into shared memory.
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnArgs p, int grid_main)
 {
+    extern __shared__ float wsm[];         // [kCombineWarps][max splits]
+    // programmatic dependent launch: start early, read partials only after the
+    // attention kernel (and everything before it) has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int s = blockIdx.x;              // segment
     const int b = s / p.Hkv, g = s % p.Hkv;
-    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, grid_main,
-                                 p.min_keys);
+    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, grid_main, p.min_keys);
     if (d.W == 0) return;
     int len;
     const int64_t s0 = seg_start(p.ctx_lens, b, g, p.Hkv, p.K, p.S_max, &len);
@@ -102,32 +110,61 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs p, int grid_
     const int c_lo = cta_of(d, s0);
     const int c_hi = cta_of(d, s0 + len - 1);
     if (c_lo == c_hi) return;              // written directly by its only CTA
+    const int n = c_hi - c_lo + 1;
 
     const int G = p.Hq / p.Hkv;
     const int rows = G * p.K;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    for (int r = blockIdx.y * nwarps + warp; r < rows; r += gridDim.y * nwarps) {
-        float M = -INFINITY;
-        for (int c = c_lo + lane; c <= c_hi; c += 32)
-            M = fmaxf(M, p.ws_lse[(size_t)(c + s) * rows + r]);
+    float *wv = wsm + warp * (grid_main + 1);
+    const int r = blockIdx.y * kCombineWarps + warp;
+    if (r >= rows) return;
+    const float *lse = p.ws_lse + (size_t)(c_lo + s) * rows + r;
+    float M = -INFINITY;
+    for (int c = lane; c < n; c += 32) M = fmaxf(M, lse[(size_t)c * rows]);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        const int i = r / G;
-        const int h = g * G + (r % G);
-        float *orow = p.out + (((size_t)b * p.K + i) * p.Hq + h) * p.D;
-        for (int dd = lane; dd < p.D; dd += 32) {
-            float acc = 0.f, wsum = 0.f;
-            for (int c = c_lo; c <= c_hi; ++c) {
-                const size_t slot = (size_t)(c + s);
-                const float lse = p.ws_lse[slot * rows + r];
-                const float w = lse == -INFINITY ? 0.f : exp2f(lse - M);
-                wsum += w;
-                acc += w * p.ws_o[(slot * rows + r) * p.D + dd];
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float wsum = 0.f;
+    for (int c = lane; c < n; c += 32) {
+        const float l = lse[(size_t)c * rows];
+        const float wc = l == -INFINITY ? 0.f : exp2f(l - M);
+        wv[c] = wc;
+        wsum += wc;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    __syncwarp();
+    const float inv = 1.f / wsum;
+    const int i = r / G;
+    const int h = g * G + (r % G);
+    float4 *orow = reinterpret_cast<float4 *>(p.out + (((size_t)b * p.K + i) * p.Hq + h) * p.D);
+    const float4 *src = reinterpret_cast<const float4 *>(p.ws_o + ((size_t)(c_lo + s) * rows + r) * p.D);
+    const size_t stride4 = (size_t)rows * p.D / 4;          // one split further
+    for (int d4 = lane; d4 < p.D / 4; d4 += 32) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int c = 0;
+        for (; c + 4 <= n; c += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = __ldcg(src + (size_t)(c + u) * stride4 + d4);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float wc = wv[c + u];
+                acc.x += wc * v[u].x;
+                acc.y += wc * v[u].y;
+                acc.z += wc * v[u].z;
+                acc.w += wc * v[u].w;
             }
-            orow[dd] = acc / wsum;
         }
+        for (; c < n; ++c) {
+            const float4 v = __ldcg(src + (size_t)c * stride4 + d4);
+            const float wc = wv[c];
+            acc.x += wc * v.x;
+            acc.y += wc * v.y;
+            acc.z += wc * v.z;
+            acc.w += wc * v.w;
+        }
+        orow[d4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
 }
 
@@ -158,10 +195,18 @@ cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st)
 cudaError_t launch_attn_combine(const AttnArgs &p, int grid_main, cudaStream_t st)
 {
     const int rows = (p.Hq / p.Hkv) * p.K;
-    const int ychunks = (rows + 7) / 8 < 16 ? (rows + 7) / 8 : 16;
-    dim3 grid(p.B * p.Hkv, ychunks);
-    attn_combine_kernel<<<grid, 256, 0, st>>>(p, grid_main);
-    return cudaGetLastError();
+    dim3 grid(p.B * p.Hkv, (rows + kCombineWarps - 1) / kCombineWarps);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kCombineWarps * 32);
+    cfg.dynamicSmemBytes = (size_t)kCombineWarps * (grid_main + 1) * sizeof(float);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_combine_kernel, p, grid_main);
 }
 
 }  // namespace orthrus

@@ -1,31 +1,46 @@
 // Tensor-core dual-view attention for sm_100a: TMA-staged bf16 K/V tiles,
-// tcgen05.mma with TMEM accumulators, one query row per softmax thread.
+// tcgen05.mma with TMEM accumulators, one query row per softmax thread, and
+// thread-block clusters that merge split-KV partials through distributed
+// shared memory.
 //
 // What it computes (Orthrus technical summary, gist.science, sections 2.2 and
 // 2.3): for one KV head g of sequence b, the G*K block queries (G query heads
 // per KV head, K block slots; row m = i*G + hl) attend over keys [0, C+K) of
 // the shared cache (DIFF, mask M_diff) or keys [0, C+i] (AR, causal within the
-// block).  Each CTA takes an equal share of the flattened key space (see
-// common.cuh) and produces, per piece, either the final rows or a split
-// partial merged by attn_combine_kernel.
+// block).
+//
+// Work split: the flattened key space of all (sequence, KV head) segments is
+// cut into equal ranges, one per CLUSTER (see common.cuh); a cluster's range
+// holds one or more pieces (segment intersections).  Inside a cluster every
+// CTA takes an equal share of each piece's 64-key boxes.  After a piece the
+// CTAs stage (row max, row sum, O) in shared memory and each merges 128/CS
+// rows across the cluster (DSMEM loads), writing either the final output
+// (cluster covers the whole segment) or one cluster partial for
+// attn_combine_kernel.
 //
 // Per 128-key tile (two 64-row TMA boxes per tensor):
 //   S  = Q K^T      tcgen05.mma kind::f16, M=128, N=64|128, K=128 (8 steps),
 //                   A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major)
 //   softmax         4 warps, thread m owns TMEM lane m: mask, running max with
 //                   lazy rescaling (threshold 2^8), exp2, row sum
-//   P = P_hi + P_lo two bf16 terms (hi = bf16(p), lo = bf16(p - hi)) written to
-//                   TMEM over the consumed S columns; the two-term split keeps
-//                   the PV product accurate to ~2^-16 relative, where a single
-//                   bf16 P (2^-9) would break the 2e-3 * RMS output tolerance
+//   P = P_hi + P_lo two bf16 terms (hi = p truncated to bf16, lo = p - hi
+//                   truncated) written to TMEM over the consumed S columns; the
+//                   two-term split keeps each weight within 2^-14 relative, where
+//                   a single bf16 P (2^-9) would break the 2e-3 * RMS tolerance
 //   O += P V        tcgen05.mma kind::f16 with A from TMEM, B = V tile (smem,
 //                   MN-major), N = 128 = head_dim, twice (hi, lo)
-// Roles: warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5 MMA issuer
+// Roles: warps 0-3 softmax + merge, warp 4 TMA producer, warp 5 MMA issuer
 // (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns) next to
-// the O accumulator (128 columns); K and V have 3-stage smem rings.
+// the O accumulator (128 columns); K and V have 3-stage smem rings; the V ring
+// doubles as the merge staging area between pieces.
+// Launched with programmatic dependent launch: barrier setup, TMEM allocation
+// and descriptor prefetch overlap the previous kernel; nothing an earlier
+// kernel may write (ctx_lens, queries, cache, workspace) is read before
+// griddepcontrol.wait.
 // Every mbarrier wait is bounded (ORTHRUS_STATUS_TIMEOUT, then drain and exit).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -35,7 +50,8 @@ namespace tc {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kStages = 3;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
 constexpr int kSBuf = 3;
 constexpr int kThreads = 192;
 constexpr int kBoxKeys = 64;
@@ -43,27 +59,38 @@ constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B = 16
 constexpr uint32_t kQBytes = 2 * kHalfBytes;            // 32 KiB
 constexpr uint32_t kStageBytes = 2 * kHalfBytes;        // 128 keys x 256 B
 constexpr uint32_t kBoxBytes = kBoxKeys * 128;          // 8 KiB (64 keys x 64 dims)
+constexpr uint32_t kStagePitch = 132;                  // floats per staged O row (conflict-free)
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kStages * kStageBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kStageBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
+constexpr uint32_t kSmemStageO = kSmemV;                  // merge receive buffer reuses the V ring
+constexpr uint32_t kSmemStageML = kSmemStageO + kRows * kStagePitch * 4;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
+static_assert(kSmemStageML + kRows * 8 <= kSmemBar, "receive buffer fits in the V ring");
+// bytes every CTA receives per piece: 128 rows (cs senders x 128/cs rows) of O and (max, sum)
+constexpr uint32_t kRecvBytes = kRows * (kD * 4 + 8);
 
 enum : int {
     B_QFULL = 0,
     B_QEMPTY,
     B_KFULL,
-    B_KEMPTY = B_KFULL + kStages,
-    B_VFULL = B_KEMPTY + kStages,
-    B_VEMPTY = B_VFULL + kStages,
-    B_SFULL = B_VEMPTY + kStages,
+    B_KEMPTY = B_KFULL + kKStages,
+    B_VFULL = B_KEMPTY + kKStages,
+    B_VEMPTY = B_VFULL + kVStages,
+    B_SFULL = B_VEMPTY + kVStages,
     B_PFULL = B_SFULL + kSBuf,
     B_PVDONE = B_PFULL + kSBuf,
     B_OFREE = B_PVDONE + kSBuf,
+    B_EPI,          // the 128 softmax threads (local, bounded)
+    B_PREADY,       // cluster: every CTA's receive buffer is free (count = cluster size)
+    B_RECV,         // local + tx: every CTA's rows for this CTA have landed
+    B_MERGED,       // local: merge finished, the V ring may be refilled
     B_DRAIN,
     B_COUNT
 };
 
 constexpr uint32_t kSmemMisc = kSmemBar + B_COUNT * 8;
+constexpr int kMaxCluster = 8;
 constexpr uint32_t kSmemUsed = kSmemMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
@@ -243,12 +270,133 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float even, float odd)
+// Packed two-lane fp32 arithmetic (one instruction for two values).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
 {
-    uint32_t d;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(odd), "f"(even));
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, C, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\tmov.b64 C, {%6, %7};\n\t"
+        "fma.rn.f32x2 D, A, B, C;\n\tmov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
 }
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "add.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "sub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Cluster-scope wait (sees writes released by other CTAs of the cluster).
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __noinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                              int32_t *status)
+{
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_cluster(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                raise_status(status, ORTHRUS_STATUS_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Generic pointer to the same shared-memory object in CTA `rank` of the cluster;
+// ordinary loads through it read that CTA's shared memory (DSMEM).
+template <typename T>
+__device__ __forceinline__ const T *map_rank(const T *p, uint32_t rank)
+{
+    unsigned long long r;
+    asm("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<unsigned long long>(p)), "r"(rank));
+    return reinterpret_cast<const T *>(r);
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Asynchronous remote stores into another CTA's shared memory; completion is
+// counted in bytes on that CTA's mbarrier.
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_async_f2(uint32_t addr, float2 v, uint32_t bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "f"(v.x), "f"(v.y), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), version 1.
@@ -269,55 +417,74 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major)
 // A piece [a, e) is read in 64-key boxes; box k starts at a + 64k except the
 // last, which is right-aligned to end at e (it may overlap the previous box or
 // start below 0, where TMA fills zeros), so no key at or past e is ever read.
+// CTA `rank` of a cluster of `cs` takes boxes [k0, k1) of the piece, two per tile.
 struct Tiling {
-    int a, e, nbox, ntile, skip;   // skip: leading rows of the last box to mask
-    __device__ __forceinline__ Tiling(int a_, int e_) : a(a_), e(e_)
+    int a, e, nbox, skip;     // skip: leading rows of the last box to mask
+    int k0, nk, ntile;
+    __device__ __forceinline__ Tiling(int a_, int e_, int rank, int cs) : a(a_), e(e_)
     {
         nbox = (e - a + kBoxKeys - 1) / kBoxKeys;
-        ntile = (nbox + 1) / 2;
         skip = a + kBoxKeys * nbox - e;
+        k0 = nbox * rank / cs;
+        nk = nbox * (rank + 1) / cs - k0;
+        ntile = (nk + 1) / 2;
     }
     __device__ __forceinline__ int box_start(int k) const
     {
         return k < nbox - 1 ? a + kBoxKeys * k : e - kBoxKeys;
     }
-    __device__ __forceinline__ int boxes_in_tile(int t) const
-    {
-        return nbox - 2 * t >= 2 ? 2 : 1;
-    }
+    __device__ __forceinline__ int boxes_in_tile(int t) const { return nk - 2 * t >= 2 ? 2 : 1; }
+    __device__ __forceinline__ int box_of(int t, int kb) const { return k0 + 2 * t + kb; }
 };
 
 struct Shared {
     uint32_t base;                 // shared address of the 1 KiB-aligned window
     volatile int *abort_flag;
+    int rank, cs;                  // cluster rank and size
     __device__ __forceinline__ uint32_t bar(int i) const { return base + kSmemBar + 8u * i; }
 };
 
 // ---------------------------------------------------------------- roles
+// Counters shared by the roles: `piece` counts every piece of the cluster's
+// range, `qp` the pieces in which this CTA has boxes (Q loads, MMAs, O use),
+// `kv`/`gt` count tiles.  Every barrier phase is awaited in order.
+
 __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                         const CUtensorMap *tq, const CUtensorMap *tk,
+                                         int cid, const CUtensorMap *tq, const CUtensorMap *tk,
                                          const CUtensorMap *tv)
 {
     const int G = p.Hq / p.Hkv;
     const uint32_t q_bytes = 2u * 128u * G * p.K;
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, blockIdx.x);
+    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t piece = 0, kv = 0;
+    uint32_t piece = 0, qp = 0, kv = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
-        if (piece > 0 && !wait_bar(sh.bar(B_QEMPTY), (piece - 1) & 1, sh.abort_flag, p.status)) {
-            ok = false;
-            break;
+        const Tiling tl(pc.a, pc.e, sh.rank, sh.cs);
+        bool merged_waited = piece == 0;
+        if (tl.ntile > 0) {
+            if (qp > 0 && !wait_bar(sh.bar(B_QEMPTY), (qp - 1) & 1, sh.abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            mbar_expect_tx(sh.bar(B_QFULL), q_bytes);
+            tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, pc.b * p.K);
+            tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, pc.b * p.K);
         }
-        mbar_expect_tx(sh.bar(B_QFULL), q_bytes);
-        tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, pc.b * p.K);
-        tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, pc.b * p.K);
-        const Tiling tl(pc.a, pc.e);
         const int z = pc.b * p.Hkv + pc.g;
         for (int t = 0; t < tl.ntile && ok; ++t, ++kv) {
             const int nb = tl.boxes_in_tile(t);
-            const uint32_t st = kv % kStages, n = kv / kStages;
             for (int which = 0; which < 2; ++which) {
+                if (which == 1 && !merged_waited) {
+                    // the V ring held the previous piece's merge staging
+                    if (!wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    merged_waited = true;
+                }
+                const uint32_t nst = which ? kVStages : kKStages;
+                const uint32_t st = kv % nst, n = kv / nst;
                 const uint32_t full = sh.bar((which ? B_VFULL : B_KFULL) + st);
                 const uint32_t empty = sh.bar((which ? B_VEMPTY : B_KEMPTY) + st);
                 if (n > 0 && !wait_bar(empty, (n - 1) & 1, sh.abort_flag, p.status)) {
@@ -328,43 +495,49 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
                 const uint32_t dst = sh.base + (which ? kSmemV : kSmemK) + st * kStageBytes;
                 const CUtensorMap *m = which ? tv : tk;
                 for (int kb = 0; kb < nb; ++kb) {
-                    const int y = tl.box_start(2 * t + kb);
+                    const int y = tl.box_start(tl.box_of(t, kb));
                     tma_load_3d(dst + kb * kBoxBytes, m, full, 0, y, z);
                     tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, m, full, 64, y, z);
                 }
             }
         }
+        if (ok && !merged_waited &&
+            !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status))
+            ok = false;
+        if (tl.ntile > 0) ++qp;
         ++piece;
     }
     if (!ok) {
         // abort: let every copy already issued land before the CTA exits
-        for (uint32_t s = 0; s < kStages; ++s) {
-            const uint32_t fills = kv / kStages + (s < kv % kStages ? 1u : 0u);
-            if (fills) {
-                wait_bar_quiet(sh.bar(B_KFULL + s), (fills - 1) & 1);
-                wait_bar_quiet(sh.bar(B_VFULL + s), (fills - 1) & 1);
-            }
+        for (uint32_t s = 0; s < kKStages; ++s) {
+            const uint32_t fills = kv / kKStages + (s < kv % kKStages ? 1u : 0u);
+            if (fills) wait_bar_quiet(sh.bar(B_KFULL + s), (fills - 1) & 1);
         }
-        if (piece > 0 || kv > 0) wait_bar_quiet(sh.bar(B_QFULL), piece & 1);
+        for (uint32_t s = 0; s < kVStages; ++s) {
+            const uint32_t fills = kv / kVStages + (s < kv % kVStages ? 1u : 0u);
+            if (fills) wait_bar_quiet(sh.bar(B_VFULL + s), (fills - 1) & 1);
+        }
+        if (qp > 0) wait_bar_quiet(sh.bar(B_QFULL), (qp - 1) & 1);
     }
 }
 
 __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                           uint32_t tmem)
+                                           int cid, uint32_t tmem)
 {
     const uint32_t idesc_pv = instr_desc(128, 128, true);
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, blockIdx.x);
+    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t piece = 0, kv = 0, gt = 0;
+    uint32_t qp = 0, kv = 0, gt = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
-        if (!wait_bar(sh.bar(B_QFULL), piece & 1, sh.abort_flag, p.status)) { ok = false; break; }
+        const Tiling tl(pc.a, pc.e, sh.rank, sh.cs);
+        if (tl.ntile == 0) continue;
+        if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
-        const Tiling tl(pc.a, pc.e);
         for (int t = 0; t <= tl.ntile && ok; ++t) {
             if (t < tl.ntile) {        // S(t) = Q K(t)^T
                 const int nb = tl.boxes_in_tile(t);
-                const uint32_t st = (kv + t) % kStages, n = (kv + t) / kStages;
+                const uint32_t st = (kv + t) % kKStages, n = (kv + t) / kKStages;
                 const uint32_t g = gt + t, buf = g % kSBuf;
                 if (!wait_bar(sh.bar(B_KFULL + st), n & 1, sh.abort_flag, p.status)) { ok = false; break; }
                 if (g >= kSBuf &&
@@ -389,15 +562,15 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
             if (t >= 1) {              // O += P(t-1) V(t-1)
                 const int tp = t - 1;
                 const int nb = tl.boxes_in_tile(tp);
-                const uint32_t st = (kv + tp) % kStages, n = (kv + tp) / kStages;
+                const uint32_t st = (kv + tp) % kVStages, n = (kv + tp) / kVStages;
                 const uint32_t g = gt + tp, buf = g % kSBuf;
                 if (!wait_bar(sh.bar(B_PFULL + buf), (g / kSBuf) & 1, sh.abort_flag, p.status) ||
                     !wait_bar(sh.bar(B_VFULL + st), n & 1, sh.abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
-                if (tp == 0 && piece > 0 &&
-                    !wait_bar(sh.bar(B_OFREE), (piece - 1) & 1, sh.abort_flag, p.status)) {
+                if (tp == 0 && qp > 0 &&
+                    !wait_bar(sh.bar(B_OFREE), (qp - 1) & 1, sh.abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
@@ -417,7 +590,7 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
         }
         kv += tl.ntile;
         gt += tl.ntile;
-        ++piece;
+        ++qp;
     }
     if (!ok) {                          // abort: wait for every MMA issued so far
         tc_commit(sh.bar(B_DRAIN));
@@ -425,8 +598,98 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     }
 }
 
-__device__ __forceinline__ void softmax_epilogue(const Shared &sh, const AttnArgs &p,
-                                                 const Decomp &d, uint32_t tmem)
+// Softmax of one S tile row (this thread's row), written back as P_hi / P_lo.
+// P_hi = p with the low 16 mantissa bits dropped (exactly a bf16 value),
+// P_lo = (p - P_hi) likewise; p - (P_hi + P_lo) < 2^-14 p.  Both halves are
+// packed two keys per 32-bit TMEM column (even key in the low half) with a
+// byte permute, so no conversion instruction is needed.
+__device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float sl2, float mb,
+                                              uint32_t p_addr)
+{
+    float2 lsum = make_float2(0.f, 0.f);
+    const float2 sc = make_float2(sl2, sl2), nm = make_float2(-mb, -mb);
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        if (ch < 2 * nb) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float2 x = ffma2(make_float2(__uint_as_float(s[32 * ch + 2 * j]),
+                                                   __uint_as_float(s[32 * ch + 2 * j + 1])),
+                                       sc, nm);
+                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                lsum = fadd2(lsum, pe);
+                const uint32_t u0 = __float_as_uint(pe.x), u1 = __float_as_uint(pe.y);
+                hi[j] = __byte_perm(u0, u1, 0x7632);
+                const float2 r = fsub2(pe, make_float2(__uint_as_float(u0 & 0xFFFF0000u),
+                                                       __uint_as_float(u1 & 0xFFFF0000u)));
+                lo[j] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+            }
+            tmem_st16(p_addr + 16 * ch, hi);
+            tmem_st16(p_addr + 64 + 16 * ch, lo);
+        }
+    }
+    return lsum.x + lsum.y;
+}
+
+// Merge rows [rank * 128/cs, (rank+1) * 128/cs) of one piece across the
+// cluster from this CTA's receive buffer (row q = sender * 128/cs + r holds
+// sender's O row and (max, sum)); write the final rows (the cluster covers the
+// whole segment) or one cluster partial (normalised O, log2-sum-exp).
+__device__ __forceinline__ void merge_rows(const AttnArgs &p, const float *recv_o, const float2 *recv_ml,
+                                           const Piece &pc, int cid, int rank, int cs, int rows, int G)
+{
+    const int rows_per = kRows / cs;                // 16..128
+    const int rr = threadIdx.x / cs;
+    const int row = rank * rows_per + rr;
+    const int cols = kD / cs;                       // floats per thread: 16..128
+    const int c0 = (threadIdx.x % cs) * cols;
+    if (row >= rows) return;
+    float wc[kMaxCluster], lc[kMaxCluster];
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+        float2 v = make_float2(-INFINITY, 0.f);
+        if (c < cs) v = recv_ml[c * rows_per + rr];
+        wc[c] = v.x;
+        lc[c] = v.y;
+        if (v.y > 0.f) M = fmaxf(M, v.x);
+    }
+    float L = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+        wc[c] = lc[c] > 0.f ? fast_exp2(wc[c] - M) : 0.f;   // weight of sender c
+        L += wc[c] * lc[c];
+    }
+    // a row can see no key of this piece (AR view, piece past C + i):
+    // zero output, zero weight in the combine
+    const float invL = L > 0.f ? 1.f / L : 0.f;
+    const bool sole = pc.a == 0 && pc.e == pc.len;
+    const size_t slot = (size_t)cid + pc.s;
+    float *dst = sole ? p.out + (((size_t)pc.b * p.K + row / G) * p.Hq + pc.g * G + row % G) * kD
+                      : p.ws_o + (slot * rows + row) * kD;
+    for (int j = 0; j < cols / 4; ++j) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c) {
+            if (c < cs && wc[c] != 0.f) {
+                const float4 v = reinterpret_cast<const float4 *>(
+                    recv_o + (c * rows_per + rr) * kStagePitch + c0)[j];
+                acc.x += wc[c] * v.x;
+                acc.y += wc[c] * v.y;
+                acc.z += wc[c] * v.z;
+                acc.w += wc[c] * v.w;
+            }
+        }
+        reinterpret_cast<float4 *>(dst + c0)[j] =
+            make_float4(acc.x * invL, acc.y * invL, acc.z * invL, acc.w * invL);
+    }
+    if (!sole && threadIdx.x % cs == 0)
+        p.ws_lse[slot * rows + row] = L > 0.f ? M + __log2f(L) : -INFINITY;
+}
+
+__device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, const AttnArgs &p,
+                                              const Decomp &d, int cid, uint32_t tmem)
 {
     const int warp = threadIdx.x >> 5;          // 0..3 = TMEM lane quarter
     const int lane = threadIdx.x & 31;
@@ -435,21 +698,31 @@ __device__ __forceinline__ void softmax_epilogue(const Shared &sh, const AttnArg
     const int rows = G * p.K;
     const bool row_ok = m < rows;
     const bool warp_ok = warp * 32 < rows;
-    const int i = m / G, hl = m % G;
+    const int i = m / G;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.scale_log2;
+    float *stage_o = reinterpret_cast<float *>(smem + kSmemStageO);
+    float2 *stage_ml = reinterpret_cast<float2 *>(smem + kSmemStageML);
+    const int cs = sh.cs, rank = sh.rank;
 
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, blockIdx.x);
+    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t piece = 0, gt = 0;
+    uint32_t gt = 0, qp = 0, piece = 0, epi = 0;
+    // all 128 softmax threads meet here; bounded, unlike a named barrier
+    auto epi_sync = [&]() -> bool {
+        mbar_arrive(sh.bar(B_EPI));
+        const bool ok = wait_bar(sh.bar(B_EPI), epi & 1, sh.abort_flag, p.status);
+        ++epi;
+        return ok;
+    };
     while (it.next(pc)) {
         const int C = pc.len - p.K;
         const int lim = p.view == ORTHRUS_AR ? C + i : 0x7FFFFFFF;   // last visible key
-        const Tiling tl(pc.a, pc.e);
+        const Tiling tl(pc.a, pc.e, rank, cs);
         float m_run = -INFINITY, l_run = 0.f;
         for (int t = 0; t < tl.ntile; ++t, ++gt) {
             const uint32_t buf = gt % kSBuf;
-            if (!wait_bar(sh.bar(B_SFULL + buf), (gt / kSBuf) & 1, sh.abort_flag, p.status)) return;
+            if (!wait_bar(sh.bar(B_SFULL + buf), (gt / kSBuf) & 1, sh.abort_flag, p.status)) return false;
             tc_fence_after();
             const int nb = tl.boxes_in_tile(t);
             if (warp_ok) {
@@ -465,29 +738,36 @@ __device__ __forceinline__ void softmax_epilogue(const Shared &sh, const AttnArg
                 int r_lo[2], r_hi[2];
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb) {
-                    const int k = 2 * t + kb;
+                    const int k = tl.box_of(t, kb);
                     const int ks = tl.box_start(k);
                     r_lo[kb] = (k == tl.nbox - 1) ? tl.skip : 0;
                     const long long hi = (long long)lim - ks;
                     r_hi[kb] = hi > 63 ? 63 : (int)hi;
                     if (!row_ok || kb >= nb) { r_lo[kb] = 64; r_hi[kb] = -1; }
                 }
-                const bool full = r_lo[0] == 0 && r_hi[0] == 63 && (nb == 1 || (r_lo[1] == 0 && r_hi[1] == 63));
-                float mx = -INFINITY;
-                if (full) {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c < 64 * nb) mx = fmaxf(mx, __uint_as_float(s[c]));
-                } else {
+                const bool full = r_lo[0] == 0 && r_hi[0] == 63 &&
+                                  (nb == 1 || (r_lo[1] == 0 && r_hi[1] == 63));
+                if (!full) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c) {
                         const int kb = c >> 6, r = c & 63;
-                        const bool v = r >= r_lo[kb] && r <= r_hi[kb];
-                        if (!v) s[c] = __float_as_uint(-INFINITY);
-                        mx = fmaxf(mx, __uint_as_float(s[c]));
+                        if (r < r_lo[kb] || r > r_hi[kb]) s[c] = __float_as_uint(-INFINITY);
                     }
                 }
-                const float m_tile = mx * sl2;
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                    mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                }
+                if (nb == 2) {
+#pragma unroll
+                    for (int c = 64; c < 128; c += 4) {
+                        mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                        mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                    }
+                }
+                const float m_tile = fmaxf(mx0, mx1) * sl2;
                 float factor = 1.f;
                 if (m_run == -INFINITY) {
                     m_run = m_tile;                       // first visible keys: O is still zero
@@ -500,7 +780,7 @@ __device__ __forceinline__ void softmax_epilogue(const Shared &sh, const AttnArg
                     // O must hold PV(t-1) before it is rescaled (t >= 1 here)
                     const uint32_t pg = gt - 1, pb = pg % kSBuf;
                     if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status))
-                        return;
+                        return false;
                     tc_fence_after();
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
@@ -513,97 +793,105 @@ __device__ __forceinline__ void softmax_epilogue(const Shared &sh, const AttnArg
                     }
                 }
                 const float mb = m_run == -INFINITY ? 0.f : m_run;
-                float lsum = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    if (ch < 2 * nb) {
-                        uint32_t hi[16], lo[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float p0 = fast_exp2(fmaf(__uint_as_float(s[32 * ch + 2 * j]), sl2, -mb));
-                            const float p1 = fast_exp2(fmaf(__uint_as_float(s[32 * ch + 2 * j + 1]), sl2, -mb));
-                            lsum += p0 + p1;
-                            const uint32_t h = pack_bf16x2(p0, p1);
-                            hi[j] = h;
-                            lo[j] = pack_bf16x2(p0 - __uint_as_float(h << 16),
-                                                p1 - __uint_as_float(h & 0xFFFF0000u));
-                        }
-                        tmem_st16(lane_base + buf * 128 + 16 * ch, hi);
-                        tmem_st16(lane_base + buf * 128 + 64 + 16 * ch, lo);
-                    }
-                }
-                l_run += lsum;
+                l_run += softmax_tile(s, nb, sl2, mb, lane_base + buf * 128);
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.bar(B_PFULL + buf));
         }
-        // epilogue: O of this piece is final once PV(last) has completed
-        {
+
+        // ---- push this CTA's (max, sum, O) rows to their owners in the cluster
+        if (tl.ntile > 0) {
             const uint32_t pg = gt - 1, pb = pg % kSBuf;
-            if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status)) return;
+            if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status)) return false;
             tc_fence_after();
         }
-        if (warp_ok) {
-            const bool sole = pc.a == 0 && pc.e == pc.len;
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            float *dst;
-            if (sole)
-                dst = p.out + (((size_t)pc.b * p.K + i) * p.Hq + pc.g * G + hl) * kD;
-            else
-                dst = p.ws_o + ((size_t)(blockIdx.x + pc.s) * rows + m) * kD;
-#pragma unroll
+        if (threadIdx.x == 0) {
+            // this CTA's V ring (the receive buffer) is idle: the piece's PVs are
+            // done and the previous merge has finished reading it
+            mbar_expect_tx(sh.bar(B_RECV), kRecvBytes);
+            fence_cluster();
+            for (int c = 0; c < cs; ++c) mbar_arrive_remote(map_shared(sh.bar(B_PREADY), c));
+        }
+        if (!wait_bar_cluster(sh.bar(B_PREADY), piece & 1, sh.abort_flag, p.status)) return false;
+        {
+            const int rows_per = kRows / cs;
+            const int owner = m / rows_per;
+            const int q = rank * rows_per + m % rows_per;
+            const uint32_t dst_o = map_shared(sh.base + kSmemStageO + q * kStagePitch * 4, owner);
+            const uint32_t dst_bar = map_shared(sh.bar(B_RECV), owner);
+            const bool have = tl.ntile > 0 && warp_ok;
+#pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t o[32];
-                tmem_ld32(lane_base + kColO + 32 * ch, o);
-                tmem_wait_ld();
-                if (row_ok) {
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * ch);
+                if (have) {
+                    tmem_ld32(lane_base + kColO + 32 * ch, o);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        d4[c] = make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
-                                            __uint_as_float(o[4 * c + 2]) * inv, __uint_as_float(o[4 * c + 3]) * inv);
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
                 }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_async_f4(dst_o + (32 * ch + 4 * c) * 4,
+                                make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
+                                            __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3])),
+                                dst_bar);
             }
-            if (row_ok && !sole)
-                p.ws_lse[(size_t)(blockIdx.x + pc.s) * rows + m] =
-                    l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+            const float2 ml = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
+                                                                      : make_float2(-INFINITY, 0.f);
+            st_async_f2(map_shared(sh.base + kSmemStageML + q * 8, owner), ml, dst_bar);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sh.bar(B_OFREE));
+        if (tl.ntile > 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sh.bar(B_OFREE));      // TMEM O may be overwritten
+            ++qp;
+        }
+        // (the expect_tx above was this CTA's one arrival; the phase completes
+        // when all kRecvBytes have landed)
+        if (!wait_bar_cluster(sh.bar(B_RECV), piece & 1, sh.abort_flag, p.status)) return false;
+
+        // ---- merge this CTA's rows across the cluster, from local shared memory
+        merge_rows(p, stage_o, stage_ml, pc, cid, rank, cs, rows, G);
+        if (!epi_sync()) return false;
+        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED));  // the V ring is free again
         ++piece;
     }
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs p)
+                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs p, int nclusters)
 {
     extern __shared__ uint8_t smem_raw[];
-    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, gridDim.x, p.min_keys);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        for (int b = 0; b < p.B; ++b)
-            if (seg_len(p.ctx_lens, b, p.K, p.S_max) == 0) raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
-    }
-    if (d.W == 0 || (int)blockIdx.x >= d.P) return;      // uniform per CTA
-
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t aligned = (raw + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (aligned - raw);
     Shared sh;
     sh.base = aligned;
     sh.abort_flag = reinterpret_cast<volatile int *>(base_ptr + kSmemMisc + 4);
+    uint32_t cs_u, cid_u;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs_u));
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(cid_u));
+    sh.cs = (int)cs_u;
+    sh.rank = (int)cluster_rank();
+    const int cid = (int)cid_u;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(base_ptr + kSmemMisc);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // ---- prologue: touches nothing an earlier kernel in the stream may write
+    pdl_trigger();
     if (threadIdx.x == 0) {
         mbar_init(sh.bar(B_QFULL), 1);
         mbar_init(sh.bar(B_QEMPTY), 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(sh.bar(B_KFULL + s), 1);
             mbar_init(sh.bar(B_KEMPTY + s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(sh.bar(B_VFULL + s), 1);
             mbar_init(sh.bar(B_VEMPTY + s), 1);
         }
@@ -613,6 +901,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(sh.bar(B_PVDONE + s), 1);
         }
         mbar_init(sh.bar(B_OFREE), 4);
+        mbar_init(sh.bar(B_EPI), 128);
+        mbar_init(sh.bar(B_PREADY), sh.cs);
+        mbar_init(sh.bar(B_RECV), 1);
+        mbar_init(sh.bar(B_MERGED), 1);
         mbar_init(sh.bar(B_DRAIN), 1);
         *sh.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -630,21 +922,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    // every CTA of the cluster has initialised its barriers before any remote arrive
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 4) {
-        softmax_epilogue(sh, p, d, tmem);
-    } else if (warp == 4) {
-        if (lane == 0) producer(sh, p, d, &tm_q, &tm_k, &tm_v);
-        __syncwarp();
-    } else {
-        if (lane == 0) mma_issuer(sh, p, d, tmem);
-        __syncwarp();
+    // ---- everything below may read what earlier kernels wrote
+    pdl_wait();
+    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, nclusters, p.min_keys);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int b = 0; b < p.B; ++b)
+            if (seg_len(p.ctx_lens, b, p.K, p.S_max) == 0) raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
+    }
+    if (d.W > 0 && cid < d.P) {                  // uniform per cluster
+        if (warp < 4) {
+            softmax_merge(sh, base_ptr, p, d, cid, tmem);
+        } else if (warp == 4) {
+            if (lane == 0) producer(sh, p, d, cid, &tm_q, &tm_k, &tm_v);
+            __syncwarp();
+        } else {
+            if (lane == 0) mma_issuer(sh, p, d, cid, tmem);
+            __syncwarp();
+        }
     }
 
     tc_fence_before();
+    __syncthreads();
+    if (*sh.abort_flag && threadIdx.x == 0) {
+        // an aborted cluster member lingers so that peers still reading its
+        // shared memory (or timing out) finish first
+        const unsigned long long t0 = global_ns();
+        while (global_ns() - t0 < 3 * kTimeoutNs) {}
+    }
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -704,8 +1013,75 @@ bool attn_tc_supported(int dtype, int D, int rows)
     return dtype == ORTHRUS_BF16 && D == tc::kD && rows <= tc::kRows && device_is_sm100();
 }
 
-cudaError_t launch_attn_tc(const AttnArgs &p, int grid, cudaStream_t st)
+namespace {
+
+struct ClusterPlan {
+    int cs = 0;          // CTAs per cluster
+    int nclusters = 0;   // co-resident clusters (the work units of the split)
+};
+
+// Cluster size and count for this device, chosen once: the largest cluster
+// size whose co-resident CTAs cover at least 85% of the SMs (fewer, larger
+// clusters mean fewer split partials), else the size with the most CTAs.
+// ORTHRUS_CLUSTER_SIZE overrides the size (1, 2, 4 or 8).
+ClusterPlan cluster_plan()
 {
+    static ClusterPlan plans[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ClusterPlan{};
+    ClusterPlan &pl = plans[dev];
+    if (pl.cs) return pl;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::kSmemAlloc) != cudaSuccess)
+        return ClusterPlan{};
+    cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    int forced = 0;
+    if (const char *env = getenv("ORTHRUS_CLUSTER_SIZE")) forced = atoi(env);
+    const int sizes[4] = {8, 4, 2, 1};
+    ClusterPlan best, most;
+    for (int cs : sizes) {
+        if (forced && cs != forced) continue;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cs * (sms / cs));
+        cfg.blockDim = dim3(tc::kThreads);
+        cfg.dynamicSmemBytes = tc::kSmemAlloc;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, tc::attn_tc_kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
+        if (n <= 0) continue;
+        if (n * cs > most.nclusters * most.cs) most = ClusterPlan{cs, n};
+        if (!best.cs && n * cs * 100 >= sms * 85) best = ClusterPlan{cs, n};
+    }
+    pl = best.cs ? best : most;
+    return pl;
+}
+
+}  // namespace
+
+bool attn_tc_plan(int *units, int *min_keys)
+{
+    const ClusterPlan pl = cluster_plan();
+    if (!pl.cs) return false;
+    *units = pl.nclusters;
+    *min_keys = 128 * pl.cs;
+    return true;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st)
+{
+    const ClusterPlan pl = cluster_plan();
+    if (!pl.cs || units < 1 || units > pl.nclusters) return cudaErrorInvalidValue;
     const int G = p.Hq / p.Hkv;
     CUtensorMap tq, tk, tv;
     const uint64_t row = tc::kD * 2;
@@ -715,17 +1091,23 @@ cudaError_t launch_attn_tc(const AttnArgs &p, int grid, cudaStream_t st)
         !encode_3d(&tv, p.v_cache, tc::kD, p.S_max, (uint64_t)p.B * p.Hkv, row,
                    (uint64_t)p.S_max * row, 64, 64, 1))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)tc::kSmemAlloc);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemAlloc, st>>>(tq, tk, tv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.cs * units);
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = tc::kSmemAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tk, tv, p, units);
     if (e != cudaSuccess) return e;
-    return launch_attn_combine(p, grid, st);
+    return launch_attn_combine(p, units, st);
 }
 
 }  // namespace orthrus

@@ -36,10 +36,11 @@ inline size_t attn_ws_bytes(int slots, int rows, int D)
 cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);
 cudaError_t launch_attn_combine(const AttnArgs &p, int grid_main, cudaStream_t st);
 
-// Tensor-core path (bf16, D == 128, G*K <= 128).  Returns cudaErrorNotSupported
-// when the device or shape does not qualify.
+// Tensor-core path (bf16, D == 128, G*K <= 128, sm_100).  attn_tc_plan gives
+// the split units (clusters) and the smallest key range worth one unit.
 bool attn_tc_supported(int dtype, int D, int rows);
-cudaError_t launch_attn_tc(const AttnArgs &p, int grid, cudaStream_t st);
+bool attn_tc_plan(int *units, int *min_keys);
+cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st);
 
 struct ConsensusArgs {
     const float *logits;
@@ -63,6 +64,7 @@ struct CommitArgs {
     int32_t *status;
     int num_layers, B, Hkv, D, S_max, K, elem_bytes;
     int copy;
+    int all_rows;        // 1: install all K block slots, no acceptance, no advance
 };
 cudaError_t launch_kv_commit(const CommitArgs &p, cudaStream_t st);
 

@@ -7,6 +7,8 @@
 //                  16-byte copies of slots 0..n_b-1 from [B, K, Hkv, D]
 //                  staging into cache rows [ctx_b, ctx_b + n_b).
 //   advance kernel one thread per sequence: ctx_b += n_b, once per step.
+// The same copy kernel, with all K slots and no advance, installs a view's
+// block K/V rows into the cache tail (orthrus_write_block).
 // The advance runs as its own launch after the copies on the same stream, so
 // every copy reads the old length.
 #include "common.cuh"
@@ -17,9 +19,15 @@ namespace orthrus {
 __device__ __forceinline__ bool commit_valid(const CommitArgs &p, int b, int *n_out,
                                              int *ctx_out)
 {
-    const int a = p.accepted[b];
     const int c = p.ctx_lens[b];
-    if (a < 0 || a > p.K || c < 0 || (int64_t)c + p.K > p.S_max) return false;
+    if (c < 0 || (int64_t)c + p.K > p.S_max) return false;
+    if (p.all_rows) {                    // block install: every slot, no acceptance
+        *n_out = p.K;
+        *ctx_out = c;
+        return true;
+    }
+    const int a = p.accepted[b];
+    if (a < 0 || a > p.K) return false;
     *n_out = a + 1 < p.K ? a + 1 : p.K;
     *ctx_out = c;
     return true;
@@ -30,7 +38,11 @@ __global__ void __launch_bounds__(256) kv_copy_kernel(CommitArgs p)
     const int layer = blockIdx.z;
     const int b = blockIdx.y;
     int n, c;
-    if (!commit_valid(p, b, &n, &c)) return;        // flagged by the advance kernel
+    if (!commit_valid(p, b, &n, &c)) {              // flagged by the advance kernel
+        if (p.all_rows && layer == 0 && blockIdx.x == 0 && threadIdx.x == 0)
+            raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
+        return;
+    }
     // 16-byte units per row and the units this sequence moves per tensor
     const int row_units = p.D * p.elem_bytes / 16;
     const int64_t units = (int64_t)n * p.Hkv * row_units;
@@ -77,6 +89,7 @@ cudaError_t launch_kv_commit(const CommitArgs &p, cudaStream_t st)
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if (p.all_rows) return cudaSuccess;            // block install never advances
     kv_advance_kernel<<<(p.B + 127) / 128, 128, 0, st>>>(p);
     return cudaGetLastError();
 }

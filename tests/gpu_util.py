@@ -21,14 +21,20 @@ def to_dev(x: np.ndarray, dtype) -> torch.Tensor:
 
 
 def run_attn(view: int, q, kc, vc, ctx, dtype, status=None, scale=0.0):
-    """Device tensors in, fp32 output tensor out (after a synchronise)."""
+    """Device tensors in, fp32 output tensor out (after a synchronise).  Without
+    a caller status word, the call must leave the device status at zero."""
     B, K, Hq, D = q.shape
     Hkv = kc.shape[1]
     out = torch.full((B, K, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
     ws = torch.empty(ob.orthrus_attn_workspace_size(B, Hq, Hkv, D, K, dtype),
                      dtype=torch.uint8, device="cuda")
+    own = status is None
+    if own:
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ob.orthrus_attn(view, q, kc, vc, ctx, out, ws, status=status, scale=scale)
     torch.cuda.synchronize()
+    if own:
+        assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
     return out
 
 

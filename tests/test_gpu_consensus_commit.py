@@ -182,3 +182,41 @@ def test_lossless_loop_on_device():
         assert int(dctx.item()) == len(seq)
     out = (seq + [anchor])[:target]
     assert out == greedy[:len(out)]
+
+
+def test_write_block_installs_every_slot_without_advancing():
+    rng = np.random.default_rng(40)
+    B, Hkv, D, K, layers = 3, 8, 128, 32, 4
+    ctx = np.array([0, 250, 1000], np.int32)
+    S = int(ctx.max()) + K
+    kcs = [rng.integers(0, 2 ** 16, size=(B, Hkv, S, D), dtype=np.uint16) for _ in range(layers)]
+    vcs = [rng.integers(0, 2 ** 16, size=(B, Hkv, S, D), dtype=np.uint16) for _ in range(layers)]
+    kbs = [rng.integers(0, 2 ** 16, size=(B, K, Hkv, D), dtype=np.uint16) for _ in range(layers)]
+    vbs = [rng.integers(0, 2 ** 16, size=(B, K, Hkv, D), dtype=np.uint16) for _ in range(layers)]
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    dk, dv, dkb, dvb = ([dev(a) for a in arrs] for arrs in (kcs, vcs, kbs, vbs))
+    dctx = torch.from_numpy(ctx).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ob.orthrus_write_block(dctx, dk, dv, dkb, dvb, status=status)
+    torch.cuda.synchronize()
+    for l in range(layers):
+        # oracle commit with a = K copies all K slots; no advance
+        oracle.kv_commit(kcs[l], vcs[l], kbs[l], vbs[l], ctx.copy(), np.full(B, K, np.int32), K,
+                         advance=False)
+        np.testing.assert_array_equal(dk[l].view(torch.int16).cpu().numpy().view(np.uint16), kcs[l])
+        np.testing.assert_array_equal(dv[l].view(torch.int16).cpu().numpy().view(np.uint16), vcs[l])
+    np.testing.assert_array_equal(dctx.cpu().numpy(), ctx)
+    assert int(status.item()) == 0
+    # a sequence without room is flagged and skipped
+    dctx2 = torch.tensor([0, S - K + 1, 5], dtype=torch.int32, device="cuda")
+    ob.orthrus_write_block(dctx2, dk[:1], dv[:1], dkb[:1], dvb[:1], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == ob.STATUS_CAPACITY
+
+
+def test_tensor_core_path_is_selected_for_bf16_d128():
+    assert ob.orthrus_attn_path(1, 32, 8, 128, 32, torch.bfloat16) == 1
+    assert ob.orthrus_attn_path(4, 32, 8, 128, 8, torch.bfloat16) == 1
+    assert ob.orthrus_attn_path(1, 16, 8, 128, 32, torch.bfloat16) == 1
+    assert ob.orthrus_attn_path(1, 16, 2, 128, 32, torch.bfloat16) == 0   # G*K = 256
+    assert ob.orthrus_attn_path(1, 4, 2, 64, 8, torch.float32) == 0
