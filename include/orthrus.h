@@ -217,6 +217,32 @@ ORTHRUS_API int orthrus_write_block(int num_layers, void *const *k_caches,
  */
 ORTHRUS_API int orthrus_attn_path(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dtype);
 
+/*
+ * orthrus_attn_static — orthrus_attn without a caller workspace, for callers
+ * that cannot allocate device memory: runtimes whose allocator belongs to
+ * another framework, engines that forbid allocation after their memory plan is
+ * fixed, or plugins that receive only input and output pointers.  (This entry
+ * point is a property of this library; the paper has no counterpart.)
+ *
+ * Same arguments and results as orthrus_attn, minus workspace and
+ * workspace_bytes.  The split-KV scratch is a fixed array inside the library
+ * of ORTHRUS_STATIC_SCRATCH_BYTES, held on every GPU that loads the library
+ * until the process exits; the call allocates and frees nothing.  Sizes whose
+ * orthrus_attn_workspace_size() exceeds that limit are rejected with
+ * ORTHRUS_ERR_WORKSPACE (bf16 attention with G*K = 128 and D = 128 fits up to
+ * about 220 (sequence, KV head) pairs on a 148-SM B200).  The first call on a
+ * device looks up the
+ * array's device address while that device is current: make it before any
+ * stream capture.  All calls share the array, which keeps the last call's
+ * contents (nothing in it needs clearing); calls that overlap on the GPU race.
+ */
+#define ORTHRUS_STATIC_SCRATCH_BYTES (16u << 20)
+ORTHRUS_API int orthrus_attn_static(orthrus_view view, orthrus_dtype dtype, const void *q,
+                                    const void *k_cache, const void *v_cache,
+                                    const int32_t *ctx_lens, int B, int Hq, int Hkv, int D,
+                                    int S_max, int K, float scale, float *out, int32_t *status,
+                                    void *stream);
+
 /* Human-readable text for an ORTHRUS_* return code (static storage). */
 ORTHRUS_API const char *orthrus_error_string(int code);
 
