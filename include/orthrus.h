@@ -80,8 +80,8 @@ typedef enum {
 /*
  * orthrus_attn_workspace_size — bytes of scratch orthrus_attn needs for these
  * sizes on the CURRENT device (the split-KV partials: one fp32 [G*K, D] tile
- * plus G*K log-sum-exp values per (CTA, KV segment) boundary).  Independent of
- * the context lengths.  Returns 0 for invalid sizes.
+ * plus G*K log-sum-exp values per (split unit, KV segment) boundary).
+ * Independent of the context lengths.  Returns 0 for invalid sizes.
  */
 ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K,
                                    orthrus_dtype dtype);

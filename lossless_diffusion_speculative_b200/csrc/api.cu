@@ -124,9 +124,9 @@ int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const vo
     a.v_cache = v_cache;
     a.ctx_lens = ctx_lens;
     a.out = out;
-    a.ws_o = static_cast<float *>(workspace);
-    size_t o_bytes = ((size_t)pl.slots * rows * D * sizeof(float) + 255) & ~(size_t)255;
-    a.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes);
+    char *ws = static_cast<char *>(workspace);
+    a.ws_o = reinterpret_cast<float *>(ws);
+    a.ws_lse = reinterpret_cast<float *>(ws + attn_ws_o_bytes(pl.slots, rows, D));
     a.status = status;
     a.B = B;
     a.Hq = Hq;

@@ -31,8 +31,8 @@
 //                   MN-major), N = 128 = head_dim, twice (hi, lo)
 // Roles: warps 0-3 softmax + merge, warp 4 TMA producer, warp 5 MMA issuer
 // (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns) next to
-// the O accumulator (128 columns); K and V have 3-stage smem rings; the V ring
-// doubles as the merge staging area between pieces.
+// the O accumulator (128 columns); K and V have 3-stage smem rings; between
+// pieces the K ring holds the outgoing rows and the V ring the incoming ones.
 // Launched with programmatic dependent launch: barrier setup, TMEM allocation
 // and descriptor prefetch overlap the previous kernel; nothing an earlier
 // kernel may write (ctx_lens, queries, cache, workspace) is read before
@@ -67,8 +67,14 @@ constexpr uint32_t kSmemStageO = kSmemV;                  // merge receive buffe
 constexpr uint32_t kSmemStageML = kSmemStageO + kRows * kStagePitch * 4;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 static_assert(kSmemStageML + kRows * 8 <= kSmemBar, "receive buffer fits in the V ring");
-// bytes every CTA receives per piece: 128 rows (cs senders x 128/cs rows) of O and (max, sum)
-constexpr uint32_t kRecvBytes = kRows * (kD * 4 + 8);
+// send buffer: this CTA's O rows and (max, sum), staged in the K ring (idle once
+// the piece's last S MMA has finished) and shipped to their owners with bulk copies
+constexpr uint32_t kSmemSendO = kSmemK;
+constexpr uint32_t kSmemSendML = kSmemSendO + kRows * kStagePitch * 4;
+static_assert(kSmemSendML + kRows * 8 <= kSmemV, "send buffer fits in the K ring");
+// bytes every CTA receives per piece: 128 rows (cs senders x 128/cs rows) of
+// padded O rows and (max, sum)
+constexpr uint32_t kRecvBytes = kRows * (kStagePitch * 4 + 8);
 
 enum : int {
     B_QFULL = 0,
@@ -84,14 +90,14 @@ enum : int {
     B_EPI,          // the 128 softmax threads (local, bounded)
     B_PREADY,       // cluster: every CTA's receive buffer is free (count = cluster size)
     B_RECV,         // local + tx: every CTA's rows for this CTA have landed
-    B_MERGED,       // local: merge finished, the V ring may be refilled
+    B_MERGED,       // local: merge finished, the K and V rings may be refilled
     B_DRAIN,
     B_COUNT
 };
 
 constexpr uint32_t kSmemMisc = kSmemBar + B_COUNT * 8;
-constexpr int kMaxCluster = 8;
-constexpr uint32_t kSmemUsed = kSmemMisc + 16;
+constexpr int kMaxCluster = kMaxSplitRanks;
+constexpr uint32_t kSmemUsed = kSmemMisc + 16;   // tmem address, abort flag, last flag
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = kSBuf * 128;                 // 384
@@ -379,21 +385,33 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
                  : "memory");
 }
 
-// Asynchronous remote stores into another CTA's shared memory; completion is
-// counted in bytes on that CTA's mbarrier.
-__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t bar)
+// Bulk copy from this CTA's shared memory into another cluster CTA's shared
+// memory; completion is counted in bytes on that CTA's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t bar_cluster)
 {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     addr),
-                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
-                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster),
+        "r"(src), "r"(bytes), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
 }
 
-__device__ __forceinline__ void st_async_f2(uint32_t addr, float2 v, uint32_t bar)
+__device__ __forceinline__ float2 lds_f2(uint32_t addr)
 {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
-                 "f"(v.x), "f"(v.y), "r"(bar)
-                 : "memory");
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
@@ -461,7 +479,11 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     bool ok = true;
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e, sh.rank, sh.cs);
-        bool merged_waited = piece == 0;
+        // the K and V rings held the previous piece's merge buffers
+        if (piece > 0 && !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
+            ok = false;
+            break;
+        }
         if (tl.ntile > 0) {
             if (qp > 0 && !wait_bar(sh.bar(B_QEMPTY), (qp - 1) & 1, sh.abort_flag, p.status)) {
                 ok = false;
@@ -475,14 +497,6 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
         for (int t = 0; t < tl.ntile && ok; ++t, ++kv) {
             const int nb = tl.boxes_in_tile(t);
             for (int which = 0; which < 2; ++which) {
-                if (which == 1 && !merged_waited) {
-                    // the V ring held the previous piece's merge staging
-                    if (!wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    merged_waited = true;
-                }
                 const uint32_t nst = which ? kVStages : kKStages;
                 const uint32_t st = kv % nst, n = kv / nst;
                 const uint32_t full = sh.bar((which ? B_VFULL : B_KFULL) + st);
@@ -501,9 +515,6 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
                 }
             }
         }
-        if (ok && !merged_waited &&
-            !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status))
-            ok = false;
         if (tl.ntile > 0) ++qp;
         ++piece;
     }
@@ -636,7 +647,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
 // cluster from this CTA's receive buffer (row q = sender * 128/cs + r holds
 // sender's O row and (max, sum)); write the final rows (the cluster covers the
 // whole segment) or one cluster partial (normalised O, log2-sum-exp).
-__device__ __forceinline__ void merge_rows(const AttnArgs &p, const float *recv_o, const float2 *recv_ml,
+__device__ __forceinline__ void merge_rows(const AttnArgs &p, uint32_t recv_o, uint32_t recv_ml,
                                            const Piece &pc, int cid, int rank, int cs, int rows, int G)
 {
     const int rows_per = kRows / cs;                // 16..128
@@ -650,7 +661,7 @@ __device__ __forceinline__ void merge_rows(const AttnArgs &p, const float *recv_
 #pragma unroll
     for (int c = 0; c < kMaxCluster; ++c) {
         float2 v = make_float2(-INFINITY, 0.f);
-        if (c < cs) v = recv_ml[c * rows_per + rr];
+        if (c < cs) v = lds_f2(recv_ml + (c * rows_per + rr) * 8);
         wc[c] = v.x;
         lc[c] = v.y;
         if (v.y > 0.f) M = fmaxf(M, v.x);
@@ -662,19 +673,20 @@ __device__ __forceinline__ void merge_rows(const AttnArgs &p, const float *recv_
         L += wc[c] * lc[c];
     }
     // a row can see no key of this piece (AR view, piece past C + i):
-    // zero output, zero weight in the combine
+    // zero output, zero weight in the final merge
     const float invL = L > 0.f ? 1.f / L : 0.f;
     const bool sole = pc.a == 0 && pc.e == pc.len;
     const size_t slot = (size_t)cid + pc.s;
     float *dst = sole ? p.out + (((size_t)pc.b * p.K + row / G) * p.Hq + pc.g * G + row % G) * kD
                       : p.ws_o + (slot * rows + row) * kD;
+    const uint32_t src0 = recv_o + (rr * kStagePitch + c0) * 4;
+    const uint32_t src_step = rows_per * kStagePitch * 4;          // next sender
     for (int j = 0; j < cols / 4; ++j) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < kMaxCluster; ++c) {
             if (c < cs && wc[c] != 0.f) {
-                const float4 v = reinterpret_cast<const float4 *>(
-                    recv_o + (c * rows_per + rr) * kStagePitch + c0)[j];
+                const float4 v = lds_f4(src0 + c * src_step + 16 * j);
                 acc.x += wc[c] * v.x;
                 acc.y += wc[c] * v.y;
                 acc.z += wc[c] * v.z;
@@ -701,8 +713,6 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
     const int i = m / G;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    float *stage_o = reinterpret_cast<float *>(smem + kSmemStageO);
-    float2 *stage_ml = reinterpret_cast<float2 *>(smem + kSmemStageML);
     const int cs = sh.cs, rank = sh.rank;
 
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
@@ -801,47 +811,32 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
             if (lane == 0) mbar_arrive(sh.bar(B_PFULL + buf));
         }
 
-        // ---- push this CTA's (max, sum, O) rows to their owners in the cluster
+        // ---- ship this CTA's (max, sum, O) rows to their owners in the cluster
         if (tl.ntile > 0) {
             const uint32_t pg = gt - 1, pb = pg % kSBuf;
             if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status)) return false;
             tc_fence_after();
         }
-        if (threadIdx.x == 0) {
-            // this CTA's V ring (the receive buffer) is idle: the piece's PVs are
-            // done and the previous merge has finished reading it
-            mbar_expect_tx(sh.bar(B_RECV), kRecvBytes);
-            fence_cluster();
-            for (int c = 0; c < cs; ++c) mbar_arrive_remote(map_shared(sh.bar(B_PREADY), c));
-        }
-        if (!wait_bar_cluster(sh.bar(B_PREADY), piece & 1, sh.abort_flag, p.status)) return false;
         {
-            const int rows_per = kRows / cs;
-            const int owner = m / rows_per;
-            const int q = rank * rows_per + m % rows_per;
-            const uint32_t dst_o = map_shared(sh.base + kSmemStageO + q * kStagePitch * 4, owner);
-            const uint32_t dst_bar = map_shared(sh.bar(B_RECV), owner);
-            const bool have = tl.ntile > 0 && warp_ok;
+            // stage into the send buffer (the K ring: the piece's S MMAs are done)
+            float *send_o = reinterpret_cast<float *>(smem + kSmemSendO);
+            float2 *send_ml = reinterpret_cast<float2 *>(smem + kSmemSendML);
+            if (tl.ntile > 0 && warp_ok) {
+                float4 *srow = reinterpret_cast<float4 *>(send_o + m * kStagePitch);
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t o[32];
-                if (have) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t o[32];
                     tmem_ld32(lane_base + kColO + 32 * ch, o);
                     tmem_wait_ld();
-                } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                    for (int c = 0; c < 8; ++c)
+                        srow[8 * ch + c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
+                                                       __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
                 }
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_async_f4(dst_o + (32 * ch + 4 * c) * 4,
-                                make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
-                                            __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3])),
-                                dst_bar);
             }
-            const float2 ml = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
-                                                                      : make_float2(-INFINITY, 0.f);
-            st_async_f2(map_shared(sh.base + kSmemStageML + q * 8, owner), ml, dst_bar);
+            send_ml[m] = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
+                                                                 : make_float2(-INFINITY, 0.f);
+            fence_proxy_async();                               // visible to the bulk copies
         }
         if (tl.ntile > 0) {
             tc_fence_before();
@@ -849,14 +844,34 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
             if (lane == 0) mbar_arrive(sh.bar(B_OFREE));      // TMEM O may be overwritten
             ++qp;
         }
+        // this CTA's V ring (the receive buffer) is idle: the piece's PVs are done
+        // and the previous merge has finished reading it
+        if (threadIdx.x == 0) mbar_expect_tx(sh.bar(B_RECV), kRecvBytes);
+        if (!epi_sync()) return false;                        // send buffer complete
+        // (each release-ordered remote arrive also orders this CTA's earlier
+        // reads of its receive buffer before the peers overwrite it)
+        if (threadIdx.x < cs) mbar_arrive_remote(map_shared(sh.bar(B_PREADY), threadIdx.x));
+        if (!wait_bar_cluster(sh.bar(B_PREADY), piece & 1, sh.abort_flag, p.status)) return false;
+        if (threadIdx.x < cs) {                               // thread o ships to owner o
+            const int o = threadIdx.x;
+            const int rows_per = kRows / cs;
+            const uint32_t bar = map_shared(sh.bar(B_RECV), o);
+            bulk_copy_to_peer(map_shared(sh.base + kSmemStageO + rank * rows_per * kStagePitch * 4, o),
+                              sh.base + kSmemSendO + o * rows_per * kStagePitch * 4,
+                              rows_per * kStagePitch * 4, bar);
+            bulk_copy_to_peer(map_shared(sh.base + kSmemStageML + rank * rows_per * 8, o),
+                              sh.base + kSmemSendML + o * rows_per * 8, rows_per * 8, bar);
+            bulk_commit();
+        }
         // (the expect_tx above was this CTA's one arrival; the phase completes
         // when all kRecvBytes have landed)
         if (!wait_bar_cluster(sh.bar(B_RECV), piece & 1, sh.abort_flag, p.status)) return false;
 
         // ---- merge this CTA's rows across the cluster, from local shared memory
-        merge_rows(p, stage_o, stage_ml, pc, cid, rank, cs, rows, G);
+        merge_rows(p, sh.base + kSmemStageO, sh.base + kSmemStageML, pc, cid, rank, cs, rows, G);
+        if (threadIdx.x < cs) bulk_wait_read();              // the send buffer has been read
         if (!epi_sync()) return false;
-        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED));  // the V ring is free again
+        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // K and V rings are free again
         ++piece;
     }
     return true;

@@ -25,12 +25,20 @@ struct AttnArgs {
     int min_keys;        // smallest key range worth a CTA
 };
 
-// Workspace layout shared by the attention paths: `slots` partial tiles.
+// Workspace layout shared by the attention paths: `slots` fp32 partial tiles
+// [rows, D], then their log2-sum-exp values [rows].
+constexpr int kMaxSplitRanks = 8;   // largest cluster the tensor-core path uses
+inline size_t attn_ws_o_bytes(int slots, int rows, int D)
+{
+    return ((size_t)slots * rows * D * sizeof(float) + 255) & ~(size_t)255;
+}
+inline size_t attn_ws_lse_bytes(int slots, int rows)
+{
+    return ((size_t)slots * rows * sizeof(float) + 255) & ~(size_t)255;
+}
 inline size_t attn_ws_bytes(int slots, int rows, int D)
 {
-    size_t o = (size_t)slots * rows * D * sizeof(float);
-    o = (o + 255) & ~(size_t)255;
-    return o + (size_t)slots * rows * sizeof(float) + 256;
+    return attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);

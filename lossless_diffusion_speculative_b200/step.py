@@ -76,7 +76,7 @@ class DecodeStep:
         self.accepted = torch.empty(B, dtype=torch.int32, device=dev)
         self.next_token = torch.empty(B, dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.attn_ws = torch.empty(ob.orthrus_attn_workspace_size(B, Hq, Hkv, D, K, dt),
+        self.attn_ws = torch.zeros(ob.orthrus_attn_workspace_size(B, Hq, Hkv, D, K, dt),
                                    dtype=torch.uint8, device=dev)
         self.cons_ws = torch.empty(ob.orthrus_consensus_workspace_size(B, K, w.vocab),
                                    dtype=torch.uint8, device=dev)

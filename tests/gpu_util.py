@@ -26,7 +26,7 @@ def run_attn(view: int, q, kc, vc, ctx, dtype, status=None, scale=0.0):
     B, K, Hq, D = q.shape
     Hkv = kc.shape[1]
     out = torch.full((B, K, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
-    ws = torch.empty(ob.orthrus_attn_workspace_size(B, Hq, Hkv, D, K, dtype),
+    ws = torch.zeros(ob.orthrus_attn_workspace_size(B, Hq, Hkv, D, K, dtype),
                      dtype=torch.uint8, device="cuda")
     own = status is None
     if own:
