@@ -32,7 +32,7 @@
 // Roles: warps 0-3 softmax + merge, warp 4 TMA producer, warp 5 MMA issuer
 // (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns) next to
 // the O accumulator (128 columns); K and V have 3-stage smem rings; between
-// pieces the K ring holds the outgoing rows and the V ring the incoming ones.
+// pieces the K ring holds the staged rows that the cluster members read.
 // Launched with programmatic dependent launch: barrier setup, TMEM allocation
 // and descriptor prefetch overlap the previous kernel; nothing an earlier
 // kernel may write (ctx_lens, queries, cache, workspace) is read before
@@ -63,18 +63,13 @@ constexpr uint32_t kStagePitch = 132;                  // floats per staged O ro
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kQBytes;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
-constexpr uint32_t kSmemStageO = kSmemV;                  // merge receive buffer reuses the V ring
-constexpr uint32_t kSmemStageML = kSmemStageO + kRows * kStagePitch * 4;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
-static_assert(kSmemStageML + kRows * 8 <= kSmemBar, "receive buffer fits in the V ring");
-// send buffer: this CTA's O rows and (max, sum), staged in the K ring (idle once
-// the piece's last S MMA has finished) and shipped to their owners with bulk copies
+// staging buffer: this CTA's O rows and (max, sum) after a piece, in the K ring
+// (idle once the piece's last S MMA has finished); the row owners read them
+// from here over distributed shared memory
 constexpr uint32_t kSmemSendO = kSmemK;
 constexpr uint32_t kSmemSendML = kSmemSendO + kRows * kStagePitch * 4;
-static_assert(kSmemSendML + kRows * 8 <= kSmemV, "send buffer fits in the K ring");
-// bytes every CTA receives per piece: 128 rows (cs senders x 128/cs rows) of
-// padded O rows and (max, sum)
-constexpr uint32_t kRecvBytes = kRows * (kStagePitch * 4 + 8);
+static_assert(kSmemSendML + kRows * 8 <= kSmemV, "staging buffer fits in the K ring");
 
 enum : int {
     B_QFULL = 0,
@@ -88,15 +83,14 @@ enum : int {
     B_PVDONE = B_PFULL + kSBuf,
     B_OFREE = B_PVDONE + kSBuf,
     B_EPI,          // the 128 softmax threads (local, bounded)
-    B_PREADY,       // cluster: every CTA's receive buffer is free (count = cluster size)
-    B_RECV,         // local + tx: every CTA's rows for this CTA have landed
-    B_MERGED,       // local: merge finished, the K and V rings may be refilled
+    B_PREADY,       // cluster: every member's rows are staged (count = cluster size)
+    B_PDONE,        // cluster: every member has read its rows from this CTA (count = cluster size)
+    B_MERGED,       // local: merge finished, the K ring may be refilled
     B_DRAIN,
     B_COUNT
 };
 
 constexpr uint32_t kSmemMisc = kSmemBar + B_COUNT * 8;
-constexpr int kMaxCluster = kMaxSplitRanks;
 constexpr uint32_t kSmemUsed = kSmemMisc + 16;   // tmem address, abort flag, last flag
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
@@ -385,37 +379,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
                  : "memory");
 }
 
-// Bulk copy from this CTA's shared memory into another cluster CTA's shared
-// memory; completion is counted in bytes on that CTA's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
-                                                  uint32_t bar_cluster)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src), "r"(bytes), "r"(bar_cluster)
-        : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ float4 lds_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ float2 lds_f2(uint32_t addr)
-{
-    float2 v;
-    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), version 1.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
@@ -609,13 +572,38 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     }
 }
 
+// 2^x for a pair of values on the FMA pipe, to take load off the MUFU unit:
+// Cody-Waite style reduction x = n + f with n = round(x) (via the 1.5 * 2^23
+// rounding constant), f in [-0.5, 0.5], and a degree-4 polynomial for 2^f fitted
+// here to minimise the relative error on that interval (max 2.7e-6, below the
+// 2^-14 of the bf16 hi/lo split of P).  The exponent is added to the result's
+// bits.  Inputs are clamped at -126 (2^-126 and below behave as 0 in the sums);
+// only used on tiles without masked keys, so no input is -inf.
+__device__ __forceinline__ float2 exp2_poly2(float2 x)
+{
+    const float kRound = 12582912.f;                 // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = fadd2(x, make_float2(kRound, kRound));
+    const float2 n = fsub2(t, make_float2(kRound, kRound));
+    const float2 f = fsub2(x, n);
+    float2 q = ffma2(make_float2(0.009569989517331123f, 0.009569989517331123f), f,
+                     make_float2(0.05591757968068123f, 0.05591757968068123f));
+    q = ffma2(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
+    q = ffma2(q, f, make_float2(0.6931218504905701f, 0.6931218504905701f));
+    q = ffma2(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Softmax of one S tile row (this thread's row), written back as P_hi / P_lo.
 // P_hi = p with the low 16 mantissa bits dropped (exactly a bf16 value),
 // P_lo = (p - P_hi) likewise; p - (P_hi + P_lo) < 2^-14 p.  Both halves are
 // packed two keys per 32-bit TMEM column (even key in the low half) with a
-// byte permute, so no conversion instruction is needed.
+// byte permute, so no conversion instruction is needed.  On tiles without
+// masked keys (`poly`, warp-uniform) one pair in four takes exp2_poly2.
 __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float sl2, float mb,
-                                              uint32_t p_addr)
+                                              uint32_t p_addr, bool poly)
 {
     float2 lsum = make_float2(0.f, 0.f);
     const float2 sc = make_float2(sl2, sl2), nm = make_float2(-mb, -mb);
@@ -628,7 +616,8 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
                 const float2 x = ffma2(make_float2(__uint_as_float(s[32 * ch + 2 * j]),
                                                    __uint_as_float(s[32 * ch + 2 * j + 1])),
                                        sc, nm);
-                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                const float2 pe = (poly && (j & 3) == 3) ? exp2_poly2(x)
+                                                         : make_float2(fast_exp2(x.x), fast_exp2(x.y));
                 lsum = fadd2(lsum, pe);
                 const uint32_t u0 = __float_as_uint(pe.x), u1 = __float_as_uint(pe.y);
                 hi[j] = __byte_perm(u0, u1, 0x7632);
@@ -643,61 +632,75 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
     return lsum.x + lsum.y;
 }
 
-// Merge rows [rank * 128/cs, (rank+1) * 128/cs) of one piece across the
-// cluster from this CTA's receive buffer (row q = sender * 128/cs + r holds
-// sender's O row and (max, sum)); write the final rows (the cluster covers the
-// whole segment) or one cluster partial (normalised O, log2-sum-exp).
-__device__ __forceinline__ void merge_rows(const AttnArgs &p, uint32_t recv_o, uint32_t recv_ml,
-                                           const Piece &pc, int cid, int rank, int cs, int rows, int G)
+// Merge rows [rank * 128/CS, (rank+1) * 128/CS) of one piece across the
+// cluster, reading every member's staged (max, sum) and O rows straight from
+// its shared memory (distributed shared memory, through generic pointers).
+// Warp w owns 32/CS consecutive rows; a row is read and written by a whole warp
+// (16 B per lane), so each staged row is one contiguous 512 B read and each
+// output row one coalesced 512 B store.  Writes the final rows (the cluster
+// covers the whole segment) or one cluster partial (normalised O and its
+// log2-sum-exp) for attn_combine_kernel.
+template <int CS>
+__device__ __forceinline__ void pull_merge(const AttnArgs &p, const float *stage_o, const float2 *stage_ml,
+                                           const Piece &pc, int cid, int rank, int rows, int G)
 {
-    const int rows_per = kRows / cs;                // 16..128
-    const int rr = threadIdx.x / cs;
-    const int row = rank * rows_per + rr;
-    const int cols = kD / cs;                       // floats per thread: 16..128
-    const int c0 = (threadIdx.x % cs) * cols;
-    if (row >= rows) return;
-    float wc[kMaxCluster], lc[kMaxCluster];
-    float M = -INFINITY;
+    constexpr int kRowsPer = kRows / CS;        // rows this CTA owns
+    constexpr int kRpw = kRowsPer / 4;          // rows per warp; kRpw * CS == 32
+    constexpr int kBatch = 16 / CS;             // rows per batch: 16 row reads in flight
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row0 = rank * kRowsPer + warp * kRpw;
+    // lane = q * CS + c holds the weight of member c for row row0 + q
+    const int my_row = row0 + lane / CS, my_src = lane % CS;
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (my_row < rows) ml = map_rank(stage_ml, my_src)[my_row];
+    float M = ml.y > 0.f ? ml.x : -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c) {
-        float2 v = make_float2(-INFINITY, 0.f);
-        if (c < cs) v = lds_f2(recv_ml + (c * rows_per + rr) * 8);
-        wc[c] = v.x;
-        lc[c] = v.y;
-        if (v.y > 0.f) M = fmaxf(M, v.x);
-    }
-    float L = 0.f;
+    for (int o = 1; o < CS; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = ml.y > 0.f ? fast_exp2(ml.x - M) : 0.f;
+    float L = w * ml.y;
 #pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c) {
-        wc[c] = lc[c] > 0.f ? fast_exp2(wc[c] - M) : 0.f;   // weight of sender c
-        L += wc[c] * lc[c];
-    }
-    // a row can see no key of this piece (AR view, piece past C + i):
-    // zero output, zero weight in the final merge
-    const float invL = L > 0.f ? 1.f / L : 0.f;
+    for (int o = 1; o < CS; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    // a row can see no key of this piece (AR view, piece past C + i): zero
+    // output, zero weight in the final merge
+    const float scale = L > 0.f ? w / L : 0.f;
     const bool sole = pc.a == 0 && pc.e == pc.len;
     const size_t slot = (size_t)cid + pc.s;
-    float *dst = sole ? p.out + (((size_t)pc.b * p.K + row / G) * p.Hq + pc.g * G + row % G) * kD
-                      : p.ws_o + (slot * rows + row) * kD;
-    const uint32_t src0 = recv_o + (rr * kStagePitch + c0) * 4;
-    const uint32_t src_step = rows_per * kStagePitch * 4;          // next sender
-    for (int j = 0; j < cols / 4; ++j) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!sole && my_src == 0 && my_row < rows)
+        p.ws_lse[slot * rows + my_row] = L > 0.f ? M + __log2f(L) : -INFINITY;
+
+    const float4 *src[CS];
 #pragma unroll
-        for (int c = 0; c < kMaxCluster; ++c) {
-            if (c < cs && wc[c] != 0.f) {
-                const float4 v = lds_f4(src0 + c * src_step + 16 * j);
-                acc.x += wc[c] * v.x;
-                acc.y += wc[c] * v.y;
-                acc.z += wc[c] * v.z;
-                acc.w += wc[c] * v.w;
+    for (int c = 0; c < CS; ++c) src[c] = reinterpret_cast<const float4 *>(map_rank(stage_o, c)) + lane;
+    constexpr int kPitch4 = kStagePitch / 4;    // float4 per staged row
+#pragma unroll
+    for (int q0 = 0; q0 < kRpw; q0 += kBatch) {
+        float4 v[kBatch][CS];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q)
+#pragma unroll
+            for (int c = 0; c < CS; ++c) v[q][c] = src[c][(row0 + q0 + q) * kPitch4];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int row = row0 + q0 + q;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < CS; ++c) {
+                // members without keys in this piece staged no O row: skip them
+                const float sc = __shfl_sync(0xffffffffu, scale, (q0 + q) * CS + c);
+                if (sc != 0.f) {
+                    acc.x = fmaf(sc, v[q][c].x, acc.x);
+                    acc.y = fmaf(sc, v[q][c].y, acc.y);
+                    acc.z = fmaf(sc, v[q][c].z, acc.z);
+                    acc.w = fmaf(sc, v[q][c].w, acc.w);
+                }
+            }
+            if (row < rows) {
+                float *dst = sole ? p.out + (((size_t)pc.b * p.K + row / G) * p.Hq + pc.g * G + row % G) * kD
+                                  : p.ws_o + (slot * rows + row) * kD;
+                reinterpret_cast<float4 *>(dst)[lane] = acc;
             }
         }
-        reinterpret_cast<float4 *>(dst + c0)[j] =
-            make_float4(acc.x * invL, acc.y * invL, acc.z * invL, acc.w * invL);
     }
-    if (!sole && threadIdx.x % cs == 0)
-        p.ws_lse[slot * rows + row] = L > 0.f ? M + __log2f(L) : -INFINITY;
 }
 
 __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, const AttnArgs &p,
@@ -764,20 +767,25 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
                         if (r < r_lo[kb] || r > r_hi[kb]) s[c] = __float_as_uint(-INFINITY);
                     }
                 }
-                float mx0 = -INFINITY, mx1 = -INFINITY;
+                float mx[8];
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                    mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; c += 16) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        mx[u] = fmax3(mx[u], __uint_as_float(s[c + 2 * u]), __uint_as_float(s[c + 2 * u + 1]));
                 }
                 if (nb == 2) {
 #pragma unroll
-                    for (int c = 64; c < 128; c += 4) {
-                        mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                        mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                    for (int c = 64; c < 128; c += 16) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            mx[u] = fmax3(mx[u], __uint_as_float(s[c + 2 * u]), __uint_as_float(s[c + 2 * u + 1]));
                     }
                 }
-                const float m_tile = fmaxf(mx0, mx1) * sl2;
+                const float m_tile =
+                    fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
                 float factor = 1.f;
                 if (m_run == -INFINITY) {
                     m_run = m_tile;                       // first visible keys: O is still zero
@@ -803,7 +811,7 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
                     }
                 }
                 const float mb = m_run == -INFINITY ? 0.f : m_run;
-                l_run += softmax_tile(s, nb, sl2, mb, lane_base + buf * 128);
+                l_run += softmax_tile(s, nb, sl2, mb, lane_base + buf * 128, __all_sync(0xffffffffu, full));
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -811,67 +819,56 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
             if (lane == 0) mbar_arrive(sh.bar(B_PFULL + buf));
         }
 
-        // ---- ship this CTA's (max, sum, O) rows to their owners in the cluster
+        // ---- stage this CTA's (max, sum, O) rows for the owners in the cluster
         if (tl.ntile > 0) {
             const uint32_t pg = gt - 1, pb = pg % kSBuf;
             if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status)) return false;
             tc_fence_after();
         }
-        {
-            // stage into the send buffer (the K ring: the piece's S MMAs are done)
-            float *send_o = reinterpret_cast<float *>(smem + kSmemSendO);
-            float2 *send_ml = reinterpret_cast<float2 *>(smem + kSmemSendML);
-            if (tl.ntile > 0 && warp_ok) {
-                float4 *srow = reinterpret_cast<float4 *>(send_o + m * kStagePitch);
+        float *stage_o = reinterpret_cast<float *>(smem + kSmemSendO);
+        float2 *stage_ml = reinterpret_cast<float2 *>(smem + kSmemSendML);
+        // (the K ring is idle: the piece's MMAs are done, and every member
+        // finished reading the previous piece's rows before B_PDONE completed)
+        if (tl.ntile > 0 && warp_ok) {
+            float4 *srow = reinterpret_cast<float4 *>(stage_o + m * kStagePitch);
 #pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + kColO + 32 * ch, o);
-                    tmem_wait_ld();
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + kColO + 32 * ch, o);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        srow[8 * ch + c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
-                                                       __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
-                }
+                for (int c = 0; c < 8; ++c)
+                    srow[8 * ch + c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
+                                                   __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
             }
-            send_ml[m] = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
-                                                                 : make_float2(-INFINITY, 0.f);
-            fence_proxy_async();                               // visible to the bulk copies
         }
+        stage_ml[m] = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
+                                                              : make_float2(-INFINITY, 0.f);
         if (tl.ntile > 0) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.bar(B_OFREE));      // TMEM O may be overwritten
             ++qp;
         }
-        // this CTA's V ring (the receive buffer) is idle: the piece's PVs are done
-        // and the previous merge has finished reading it
-        if (threadIdx.x == 0) mbar_expect_tx(sh.bar(B_RECV), kRecvBytes);
-        if (!epi_sync()) return false;                        // send buffer complete
-        // (each release-ordered remote arrive also orders this CTA's earlier
-        // reads of its receive buffer before the peers overwrite it)
+        if (!epi_sync()) return false;                        // staging complete
+        // release-ordered remote arrives: every member's staged rows are
+        // visible once B_PREADY completes
         if (threadIdx.x < cs) mbar_arrive_remote(map_shared(sh.bar(B_PREADY), threadIdx.x));
         if (!wait_bar_cluster(sh.bar(B_PREADY), piece & 1, sh.abort_flag, p.status)) return false;
-        if (threadIdx.x < cs) {                               // thread o ships to owner o
-            const int o = threadIdx.x;
-            const int rows_per = kRows / cs;
-            const uint32_t bar = map_shared(sh.bar(B_RECV), o);
-            bulk_copy_to_peer(map_shared(sh.base + kSmemStageO + rank * rows_per * kStagePitch * 4, o),
-                              sh.base + kSmemSendO + o * rows_per * kStagePitch * 4,
-                              rows_per * kStagePitch * 4, bar);
-            bulk_copy_to_peer(map_shared(sh.base + kSmemStageML + rank * rows_per * 8, o),
-                              sh.base + kSmemSendML + o * rows_per * 8, rows_per * 8, bar);
-            bulk_commit();
-        }
-        // (the expect_tx above was this CTA's one arrival; the phase completes
-        // when all kRecvBytes have landed)
-        if (!wait_bar_cluster(sh.bar(B_RECV), piece & 1, sh.abort_flag, p.status)) return false;
 
-        // ---- merge this CTA's rows across the cluster, from local shared memory
-        merge_rows(p, sh.base + kSmemStageO, sh.base + kSmemStageML, pc, cid, rank, cs, rows, G);
-        if (threadIdx.x < cs) bulk_wait_read();              // the send buffer has been read
-        if (!epi_sync()) return false;
-        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // K and V rings are free again
+        // ---- merge this CTA's rows across the cluster
+        switch (cs) {
+        case 1: pull_merge<1>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
+        case 2: pull_merge<2>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
+        case 4: pull_merge<4>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
+        default: pull_merge<8>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
+        }
+        if (!epi_sync()) return false;                        // this CTA's reads are done
+        if (threadIdx.x < cs) mbar_arrive_remote(map_shared(sh.bar(B_PDONE), threadIdx.x));
+        // nobody reads this CTA's staging buffer any more: the K ring may be
+        // refilled (and the CTA may exit)
+        if (!wait_bar_cluster(sh.bar(B_PDONE), piece & 1, sh.abort_flag, p.status)) return false;
+        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED));
         ++piece;
     }
     return true;
@@ -918,7 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(sh.bar(B_OFREE), 4);
         mbar_init(sh.bar(B_EPI), 128);
         mbar_init(sh.bar(B_PREADY), sh.cs);
-        mbar_init(sh.bar(B_RECV), 1);
+        mbar_init(sh.bar(B_PDONE), sh.cs);
         mbar_init(sh.bar(B_MERGED), 1);
         mbar_init(sh.bar(B_DRAIN), 1);
         *sh.abort_flag = 0;
