@@ -79,9 +79,10 @@ typedef enum {
 
 /*
  * orthrus_attn_workspace_size — bytes of scratch orthrus_attn needs for these
- * sizes on the CURRENT device (the split-KV partials: one fp32 [G*K, D] tile
- * plus G*K log-sum-exp values per (split unit, KV segment) boundary).
- * Independent of the context lengths.  Returns 0 for invalid sizes.
+ * sizes on the CURRENT device (a 1280-byte block of split-merge counters, then
+ * the split-KV partials: one fp32 [G*K, D] tile plus G*K log-sum-exp values
+ * per (split unit, KV segment) boundary).  Independent of the context
+ * lengths.  Returns 0 for invalid sizes.
  */
 ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K,
                                    orthrus_dtype dtype);
@@ -111,8 +112,12 @@ ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, in
  *   scale     softmax scale; <= 0 selects 1/sqrt(D).
  *   out       [B, K, Hq, D] fp32.
  *   workspace device scratch of at least orthrus_attn_workspace_size() bytes,
- *             16-byte aligned; contents need no initialisation and are
- *             clobbered.  Calls that overlap on the device must not share it.
+ *             16-byte aligned.  Zero-fill it once before its first use
+ *             (cudaMemset): its leading counter block must be zero when a call
+ *             starts, and every call that completes leaves it zero again (the
+ *             rest is scratch, clobbered).  A call that ended with
+ *             ORTHRUS_STATUS_TIMEOUT may leave counters set: zero it again.
+ *             Calls that overlap on the device must not share it.
  *   status    optional device int32 (see ORTHRUS_STATUS_*).  A sequence whose
  *             ctx_lens[b] is negative or leaves no room for the block
  *             (ctx_lens[b] + K > S_max) sets ORTHRUS_STATUS_CAPACITY and its
@@ -230,11 +235,13 @@ ORTHRUS_API int orthrus_attn_path(int B, int Hq, int Hkv, int D, int K, orthrus_
  * until the process exits; the call allocates and frees nothing.  Sizes whose
  * orthrus_attn_workspace_size() exceeds that limit are rejected with
  * ORTHRUS_ERR_WORKSPACE (bf16 attention with G*K = 128 and D = 128 fits up to
- * about 220 (sequence, KV head) pairs on a 148-SM B200).  The first call on a
+ * about 100 (sequence, KV head) pairs on a 148-SM B200).  The first call on a
  * device looks up the
  * array's device address while that device is current: make it before any
- * stream capture.  All calls share the array, which keeps the last call's
- * contents (nothing in it needs clearing); calls that overlap on the GPU race.
+ * stream capture.  All calls share the array, which starts zeroed and is left
+ * as orthrus_attn requires of a workspace by every call that completes (a
+ * call that timed out may leave it unusable for the rest of the process);
+ * calls that overlap on the GPU race.
  */
 #define ORTHRUS_STATIC_SCRATCH_BYTES (16u << 20)
 ORTHRUS_API int orthrus_attn_static(orthrus_view view, orthrus_dtype dtype, const void *q,

@@ -48,8 +48,7 @@ bool attn_shape_supported(int Hq, int Hkv, int D, int K)
            (int64_t)(Hq / Hkv) * K <= 4096;
 }
 
-// `grid` is the number of split units: CTAs on the CUDA-core path, clusters on
-// the tensor-core path.
+// `grid` is the number of split units (CTAs).
 AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dt, int sms)
 {
     AttnPlan pl;
@@ -125,8 +124,9 @@ int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const vo
     a.ctx_lens = ctx_lens;
     a.out = out;
     char *ws = static_cast<char *>(workspace);
-    a.ws_o = reinterpret_cast<float *>(ws);
-    a.ws_lse = reinterpret_cast<float *>(ws + attn_ws_o_bytes(pl.slots, rows, D));
+    a.ws_sync = reinterpret_cast<int32_t *>(ws);
+    a.ws_o = reinterpret_cast<float *>(ws + kSyncBytes);
+    a.ws_lse = reinterpret_cast<float *>(ws + kSyncBytes + attn_ws_o_bytes(pl.slots, rows, D));
     a.status = status;
     a.B = B;
     a.Hq = Hq;

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs p)
 #pragma unroll
                 for (int t = 0; t < DPL; ++t) orow[lane + 32 * t] = o[t] * inv;
                 if (lane == 0)
-                    p.ws_lse[(size_t)slot * rows + r] = l > 0.f ? m + log2f(l) : -INFINITY;
+                    p.ws_lse[(size_t)slot * lse_pitch(rows) + r] = l > 0.f ? m + log2f(l) : -INFINITY;
             }
         }
     }
@@ -119,14 +119,15 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
     float *wv = wsm + warp * (grid_main + 1);
     const int r = blockIdx.y * kCombineWarps + warp;
     if (r >= rows) return;
-    const float *lse = p.ws_lse + (size_t)(c_lo + s) * rows + r;
+    const int lp = lse_pitch(rows);
+    const float *lse = p.ws_lse + (size_t)(c_lo + s) * lp + r;
     float M = -INFINITY;
-    for (int c = lane; c < n; c += 32) M = fmaxf(M, lse[(size_t)c * rows]);
+    for (int c = lane; c < n; c += 32) M = fmaxf(M, lse[(size_t)c * lp]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float wsum = 0.f;
     for (int c = lane; c < n; c += 32) {
-        const float l = lse[(size_t)c * rows];
+        const float l = lse[(size_t)c * lp];
         const float wc = l == -INFINITY ? 0.f : exp2f(l - M);
         wv[c] = wc;
         wsum += wc;

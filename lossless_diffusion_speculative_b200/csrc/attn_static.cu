@@ -12,9 +12,10 @@
 // every GPU that loads the library holds it until the process exits.  Its
 // device address is looked up once per device, on the first call made while
 // that device is current (cudaGetSymbolAddress), so make the first call on each
-// device before any stream capture.  All calls share the one array and it keeps
-// the last call's contents; nothing in it needs to start at zero (each call
-// writes every scratch value it reads).  Calls that overlap on the GPU (other
+// device before any stream capture.  All calls share the one array; it starts
+// zeroed (a __device__ array is zero-initialised when the module loads), which
+// is what orthrus_attn needs of a fresh workspace, and every completed call
+// leaves its counter block zero again.  Calls that overlap on the GPU (other
 // streams, other host threads) race on the array.
 #include <mutex>
 

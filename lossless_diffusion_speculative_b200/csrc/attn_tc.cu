@@ -1,7 +1,6 @@
 // Tensor-core dual-view attention for sm_100a: TMA-staged bf16 K/V tiles,
 // tcgen05.mma with TMEM accumulators, one query row per softmax thread, and
-// thread-block clusters that merge split-KV partials through distributed
-// shared memory.
+// split-KV partials merged inside the kernel (one launch per call).
 //
 // What it computes (Orthrus technical summary, gist.science, sections 2.2 and
 // 2.3): for one KV head g of sequence b, the G*K block queries (G query heads
@@ -10,13 +9,13 @@
 // block).
 //
 // Work split: the flattened key space of all (sequence, KV head) segments is
-// cut into equal ranges, one per CLUSTER (see common.cuh); a cluster's range
-// holds one or more pieces (segment intersections).  Inside a cluster every
-// CTA takes an equal share of each piece's 64-key boxes.  After a piece the
-// CTAs stage (row max, row sum, O) in shared memory and each merges 128/CS
-// rows across the cluster (DSMEM loads), writing either the final output
-// (cluster covers the whole segment) or one cluster partial for
-// attn_combine_kernel.
+// cut into equal ranges, one per CTA (one CTA per SM, see common.cuh); a CTA's
+// range holds one or more pieces (segment intersections).  After a piece the
+// softmax warps write its rows, normalised by the row sum: the final output
+// when the CTA covers the whole segment, else one split partial (with its
+// log2-sum-exp).  After its last piece a CTA that shares a segment waits for
+// the segment's other CTAs (a counter in the workspace; all CTAs are resident,
+// one per SM) and merges its share of the segment's rows.
 //
 // Per 128-key tile (two 64-row TMA boxes per tensor):
 //   S  = Q K^T      tcgen05.mma kind::f16, M=128, N=64|128, K=128 (8 steps),
@@ -29,10 +28,10 @@
 //                   a single bf16 P (2^-9) would break the 2e-3 * RMS tolerance
 //   O += P V        tcgen05.mma kind::f16 with A from TMEM, B = V tile (smem,
 //                   MN-major), N = 128 = head_dim, twice (hi, lo)
-// Roles: warps 0-3 softmax + merge, warp 4 TMA producer, warp 5 MMA issuer
-// (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns) next to
-// the O accumulator (128 columns); K and V have 3-stage smem rings; between
-// pieces the K ring holds the staged rows that the cluster members read.
+// Roles: warps 0-3 softmax + output rows, warp 4 TMA producer, warp 5 MMA
+// issuer (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns)
+// next to the O accumulator (128 columns); K and V have 3-stage smem rings;
+// after a piece the K ring stages the output rows for their bulk copies.
 // Launched with programmatic dependent launch: barrier setup, TMEM allocation
 // and descriptor prefetch overlap the previous kernel; nothing an earlier
 // kernel may write (ctx_lens, queries, cache, workspace) is read before
@@ -64,12 +63,19 @@ constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kQBytes;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
-// staging buffer: this CTA's O rows and (max, sum) after a piece, in the K ring
-// (idle once the piece's last S MMA has finished); the row owners read them
-// from here over distributed shared memory
-constexpr uint32_t kSmemSendO = kSmemK;
-constexpr uint32_t kSmemSendML = kSmemSendO + kRows * kStagePitch * 4;
-static_assert(kSmemSendML + kRows * 8 <= kSmemV, "staging buffer fits in the K ring");
+// staging rows for the output bulk copies after a piece, in the K ring (idle
+// once the piece's last S MMA has finished); the padded pitch keeps the
+// row-per-thread writes free of bank conflicts
+constexpr uint32_t kSmemStage = kSmemK;
+static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemV, "staging rows fit in the K ring");
+// split merge, after the last piece, over the idle K and V rings: the
+// gathered partial rows (n x nr rows of D floats, n * nr < rows + n <= 128 +
+// kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
+// one weight row per warp (4 x n floats)
+constexpr uint32_t kSmemGather = kSmemK;
+static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
+                      4 * kMaxSyncUnits * 4 <= kSmemBar,
+              "split merge fits in the rings");
 
 enum : int {
     B_QFULL = 0,
@@ -83,15 +89,16 @@ enum : int {
     B_PVDONE = B_PFULL + kSBuf,
     B_OFREE = B_PVDONE + kSBuf,
     B_EPI,          // the 128 softmax threads (local, bounded)
-    B_PREADY,       // cluster: every member's rows are staged (count = cluster size)
-    B_PDONE,        // cluster: every member has read its rows from this CTA (count = cluster size)
-    B_MERGED,       // local: merge finished, the K ring may be refilled
+    B_MERGED,       // the piece's rows are out: the K ring may be refilled
+    B_GATHER,       // tx: the split partials of a segment have landed in smem
     B_DRAIN,
     B_COUNT
 };
 
 constexpr uint32_t kSmemMisc = kSmemBar + B_COUNT * 8;
-constexpr uint32_t kSmemUsed = kSmemMisc + 16;   // tmem address, abort flag, last flag
+// (after tmem address and abort flag) the split (W, P) and 2 shared pieces
+constexpr uint32_t kSmemPend = kSmemMisc + 16;
+constexpr uint32_t kSmemUsed = kSmemPend + 16 + 2 * 32;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = kSBuf * 128;                 // 384
@@ -304,6 +311,17 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b)
     return d;
 }
 
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "mul.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
     float d;
@@ -317,66 +335,51 @@ __device__ __forceinline__ void pdl_trigger()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Cluster-scope wait (sees writes released by other CTAs of the cluster).
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity)
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to
+// global memory, tracked by the issuing thread's bulk-async group.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes)
 {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __noinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                              int32_t *status)
-{
-    const unsigned long long t0 = global_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_cluster(bar, parity)) return true;
-        if ((it & 63u) == 63u) {
-            if (*abort_flag) return false;
-            if (global_ns() - t0 > kTimeoutNs) {
-                *abort_flag = 1;
-                raise_status(status, ORTHRUS_STATUS_TIMEOUT);
-                return false;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ uint32_t cluster_rank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address of the same shared-memory offset in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_shared(uint32_t addr, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-
-// Generic pointer to the same shared-memory object in CTA `rank` of the cluster;
-// ordinary loads through it read that CTA's shared memory (DSMEM).
-template <typename T>
-__device__ __forceinline__ const T *map_rank(const T *p, uint32_t rank)
-{
-    unsigned long long r;
-    asm("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<unsigned long long>(p)), "r"(rank));
-    return reinterpret_cast<const T *>(r);
-}
-
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<unsigned long long>(dst)),
+                 "r"(src), "r"(bytes)
                  : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of this thread's bulk copies may be overwritten
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's bulk copies are complete (their writes performed)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy writes to shared memory become visible to the async proxy
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// the same between the async proxy's and generic accesses to global memory
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Bulk copy of `bytes` (multiple of 16) from global to this CTA's shared
+// memory; completion is counted in bytes on mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst),
+                 "l"(reinterpret_cast<unsigned long long>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Split-merge counters in global memory (device scope).
+__device__ __forceinline__ void counter_add_release(int32_t *c, int32_t v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(c), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t counter_load_acquire(const int32_t *c)
+{
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    return v;
+}
+__device__ __forceinline__ int32_t counter_fetch_add_acq_rel(int32_t *c, int32_t v)
+{
+    int32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(c), "r"(v) : "memory");
+    return old;
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -398,37 +401,46 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major)
 // A piece [a, e) is read in 64-key boxes; box k starts at a + 64k except the
 // last, which is right-aligned to end at e (it may overlap the previous box or
 // start below 0, where TMA fills zeros), so no key at or past e is ever read.
-// CTA `rank` of a cluster of `cs` takes boxes [k0, k1) of the piece, two per tile.
+// Tiles take the boxes two at a time (the last tile may hold one).
 struct Tiling {
     int a, e, nbox, skip;     // skip: leading rows of the last box to mask
-    int k0, nk, ntile;
-    __device__ __forceinline__ Tiling(int a_, int e_, int rank, int cs) : a(a_), e(e_)
+    int ntile;
+    __device__ __forceinline__ Tiling(int a_, int e_) : a(a_), e(e_)
     {
         nbox = (e - a + kBoxKeys - 1) / kBoxKeys;
         skip = a + kBoxKeys * nbox - e;
-        k0 = nbox * rank / cs;
-        nk = nbox * (rank + 1) / cs - k0;
-        ntile = (nk + 1) / 2;
+        ntile = (nbox + 1) / 2;
     }
     __device__ __forceinline__ int box_start(int k) const
     {
         return k < nbox - 1 ? a + kBoxKeys * k : e - kBoxKeys;
     }
-    __device__ __forceinline__ int boxes_in_tile(int t) const { return nk - 2 * t >= 2 ? 2 : 1; }
-    __device__ __forceinline__ int box_of(int t, int kb) const { return k0 + 2 * t + kb; }
+    __device__ __forceinline__ int boxes_in_tile(int t) const { return nbox - 2 * t >= 2 ? 2 : 1; }
+    __device__ __forceinline__ int box_of(int t, int kb) const { return 2 * t + kb; }
+};
+
+// A segment shared with other CTAs: the n CTAs [c_lo, c_lo + n) hold its
+// partials in workspace slots c_lo + s, ..., c_lo + n - 1 + s.
+struct SplitInfo {
+    int b, g, s, c_lo, n;
+};
+// What the epilogue records of a shared piece (in shared memory, so that
+// nothing stays live in registers across the tile loop).
+struct SharedPiece {
+    int64_t s0;
+    int b, g, s, len;
 };
 
 struct Shared {
     uint32_t base;                 // shared address of the 1 KiB-aligned window
     volatile int *abort_flag;
-    int rank, cs;                  // cluster rank and size
     __device__ __forceinline__ uint32_t bar(int i) const { return base + kSmemBar + 8u * i; }
 };
 
 // ---------------------------------------------------------------- roles
-// Counters shared by the roles: `piece` counts every piece of the cluster's
-// range, `qp` the pieces in which this CTA has boxes (Q loads, MMAs, O use),
-// `kv`/`gt` count tiles.  Every barrier phase is awaited in order.
+// Counters shared by the roles: `piece`/`qp` count the pieces of the CTA's
+// range (Q loads, MMAs, O use), `kv`/`gt` count tiles.  Every barrier phase
+// is awaited in order.
 
 __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
                                          int cid, const CUtensorMap *tq, const CUtensorMap *tk,
@@ -441,7 +453,7 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     uint32_t piece = 0, qp = 0, kv = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
-        const Tiling tl(pc.a, pc.e, sh.rank, sh.cs);
+        const Tiling tl(pc.a, pc.e);
         // the K and V rings held the previous piece's merge buffers
         if (piece > 0 && !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
             ok = false;
@@ -504,7 +516,7 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     uint32_t qp = 0, kv = 0, gt = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
-        const Tiling tl(pc.a, pc.e, sh.rank, sh.cs);
+        const Tiling tl(pc.a, pc.e);
         if (tl.ntile == 0) continue;
         if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -572,38 +584,13 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     }
 }
 
-// 2^x for a pair of values on the FMA pipe, to take load off the MUFU unit:
-// Cody-Waite style reduction x = n + f with n = round(x) (via the 1.5 * 2^23
-// rounding constant), f in [-0.5, 0.5], and a degree-4 polynomial for 2^f fitted
-// here to minimise the relative error on that interval (max 2.7e-6, below the
-// 2^-14 of the bf16 hi/lo split of P).  The exponent is added to the result's
-// bits.  Inputs are clamped at -126 (2^-126 and below behave as 0 in the sums);
-// only used on tiles without masked keys, so no input is -inf.
-__device__ __forceinline__ float2 exp2_poly2(float2 x)
-{
-    const float kRound = 12582912.f;                 // 1.5 * 2^23
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
-    const float2 t = fadd2(x, make_float2(kRound, kRound));
-    const float2 n = fsub2(t, make_float2(kRound, kRound));
-    const float2 f = fsub2(x, n);
-    float2 q = ffma2(make_float2(0.009569989517331123f, 0.009569989517331123f), f,
-                     make_float2(0.05591757968068123f, 0.05591757968068123f));
-    q = ffma2(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
-    q = ffma2(q, f, make_float2(0.6931218504905701f, 0.6931218504905701f));
-    q = ffma2(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Softmax of one S tile row (this thread's row), written back as P_hi / P_lo.
 // P_hi = p with the low 16 mantissa bits dropped (exactly a bf16 value),
 // P_lo = (p - P_hi) likewise; p - (P_hi + P_lo) < 2^-14 p.  Both halves are
 // packed two keys per 32-bit TMEM column (even key in the low half) with a
-// byte permute, so no conversion instruction is needed.  On tiles without
-// masked keys (`poly`, warp-uniform) one pair in four takes exp2_poly2.
+// byte permute, so no conversion instruction is needed.
 __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float sl2, float mb,
-                                              uint32_t p_addr, bool poly)
+                                              uint32_t p_addr)
 {
     float2 lsum = make_float2(0.f, 0.f);
     const float2 sc = make_float2(sl2, sl2), nm = make_float2(-mb, -mb);
@@ -616,8 +603,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
                 const float2 x = ffma2(make_float2(__uint_as_float(s[32 * ch + 2 * j]),
                                                    __uint_as_float(s[32 * ch + 2 * j + 1])),
                                        sc, nm);
-                const float2 pe = (poly && (j & 3) == 3) ? exp2_poly2(x)
-                                                         : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                 lsum = fadd2(lsum, pe);
                 const uint32_t u0 = __float_as_uint(pe.x), u1 = __float_as_uint(pe.y);
                 hi[j] = __byte_perm(u0, u1, 0x7632);
@@ -632,79 +618,103 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
     return lsum.x + lsum.y;
 }
 
-// Merge rows [rank * 128/CS, (rank+1) * 128/CS) of one piece across the
-// cluster, reading every member's staged (max, sum) and O rows straight from
-// its shared memory (distributed shared memory, through generic pointers).
-// Warp w owns 32/CS consecutive rows; a row is read and written by a whole warp
-// (16 B per lane), so each staged row is one contiguous 512 B read and each
-// output row one coalesced 512 B store.  Writes the final rows (the cluster
-// covers the whole segment) or one cluster partial (normalised O and its
-// log2-sum-exp) for attn_combine_kernel.
-template <int CS>
-__device__ __forceinline__ void pull_merge(const AttnArgs &p, const float *stage_o, const float2 *stage_ml,
-                                           const Piece &pc, int cid, int rank, int rows, int G)
+// Merge of one shared segment, by CTA cid (see softmax_epilogue).  Thread 0
+// waits until all n CTAs have published; warp 0 then gathers this CTA's share
+// of the rows of all n partials, with their log2-sum-exp values, into shared
+// memory (lane q issues the bulk copies of partial q), and thread 0 leaves
+// (depart[c_lo] += 1; the last to leave resets both counters).  Each warp then
+// merges whole rows: lanes compute the weights 2^(lse_q - max) / sum of the
+// row's partials (the log-sum-exp merge of flash-decoding), then lane c4
+// accumulates 16-byte column c4 over the partials and stores it.
+// Returns the B_GATHER phases used (0 or 1), or -1 after an abort.
+__device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag, uint8_t *smem,
+                                        int32_t *ws_sync, const float *ws_o, const float *ws_lse,
+                                        float *out, int32_t *status, SplitInfo sp, int cid, int rows,
+                                        int G, int K, int Hq, uint32_t gph)
 {
-    constexpr int kRowsPer = kRows / CS;        // rows this CTA owns
-    constexpr int kRpw = kRowsPer / 4;          // rows per warp; kRpw * CS == 32
-    constexpr int kBatch = 16 / CS;             // rows per batch: 16 row reads in flight
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row0 = rank * kRowsPer + warp * kRpw;
-    // lane = q * CS + c holds the weight of member c for row row0 + q
-    const int my_row = row0 + lane / CS, my_src = lane % CS;
-    float2 ml = make_float2(-INFINITY, 0.f);
-    if (my_row < rows) ml = map_rank(stage_ml, my_src)[my_row];
-    float M = ml.y > 0.f ? ml.x : -INFINITY;
-#pragma unroll
-    for (int o = 1; o < CS; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = ml.y > 0.f ? fast_exp2(ml.x - M) : 0.f;
-    float L = w * ml.y;
-#pragma unroll
-    for (int o = 1; o < CS; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    // a row can see no key of this piece (AR view, piece past C + i): zero
-    // output, zero weight in the final merge
-    const float scale = L > 0.f ? w / L : 0.f;
-    const bool sole = pc.a == 0 && pc.e == pc.len;
-    const size_t slot = (size_t)cid + pc.s;
-    if (!sole && my_src == 0 && my_row < rows)
-        p.ws_lse[slot * rows + my_row] = L > 0.f ? M + __log2f(L) : -INFINITY;
-
-    const float4 *src[CS];
-#pragma unroll
-    for (int c = 0; c < CS; ++c) src[c] = reinterpret_cast<const float4 *>(map_rank(stage_o, c)) + lane;
-    constexpr int kPitch4 = kStagePitch / 4;    // float4 per staged row
-#pragma unroll
-    for (int q0 = 0; q0 < kRpw; q0 += kBatch) {
-        float4 v[kBatch][CS];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q)
-#pragma unroll
-            for (int c = 0; c < CS; ++c) v[q][c] = src[c][(row0 + q0 + q) * kPitch4];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int row = row0 + q0 + q;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < CS; ++c) {
-                // members without keys in this piece staged no O row: skip them
-                const float sc = __shfl_sync(0xffffffffu, scale, (q0 + q) * CS + c);
-                if (sc != 0.f) {
-                    acc.x = fmaf(sc, v[q][c].x, acc.x);
-                    acc.y = fmaf(sc, v[q][c].y, acc.y);
-                    acc.z = fmaf(sc, v[q][c].z, acc.z);
-                    acc.w = fmaf(sc, v[q][c].w, acc.w);
+    const uint32_t bar = base + kSmemBar + 8u * B_GATHER;
+    const int lp = lse_pitch(rows);
+    const int j = cid - sp.c_lo;
+    const int r_lo = j * rows / sp.n, nr = (j + 1) * rows / sp.n - r_lo;
+    const int l_lo = r_lo & ~3, nl = ((r_lo + nr + 3) & ~3) - l_lo;   // 16-byte lse rows
+    const uint32_t o_bytes = (uint32_t)nr * kD * 4, l_bytes = (uint32_t)nl * 4;
+    const uint32_t s_lse = kSmemGather + (uint32_t)sp.n * o_bytes;     // after the O rows
+    const uint32_t s_w = s_lse + (((uint32_t)sp.n * l_bytes + 15u) & ~15u);   // [4 warps][n] weights
+    int32_t *arrive = ws_sync + sp.c_lo;
+    if (warp == 0) {
+        bool ok = true;
+        if (lane == 0) {
+            const unsigned long long t0 = global_ns();
+            while (counter_load_acquire(arrive) < sp.n) {
+                if (*abort_flag || global_ns() - t0 > kTimeoutNs) {
+                    *abort_flag = 1;
+                    raise_status(status, ORTHRUS_STATUS_TIMEOUT);
+                    ok = false;
+                    break;
                 }
             }
-            if (row < rows) {
-                float *dst = sole ? p.out + (((size_t)pc.b * p.K + row / G) * p.Hq + pc.g * G + row % G) * kD
-                                  : p.ws_o + (slot * rows + row) * kD;
-                reinterpret_cast<float4 *>(dst)[lane] = acc;
+            if (ok && nr > 0) mbar_expect_tx(bar, (uint32_t)sp.n * (o_bytes + l_bytes));
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) return -1;
+        // (lane 0's acquire covers the warp: __syncwarp orders the lanes after
+        // it, and the proxy fence orders the bulk reads after both)
+        __syncwarp();
+        fence_proxy_async_global();
+        if (nr > 0)
+            for (int q = lane; q < sp.n; q += 32) {
+                const size_t slot = (size_t)sp.c_lo + q + sp.s;
+                bulk_load(base + kSmemGather + q * o_bytes, ws_o + (slot * rows + r_lo) * kD, o_bytes, bar);
+                bulk_load(base + s_lse + q * l_bytes, ws_lse + slot * lp + l_lo, l_bytes, bar);
             }
+        if (lane == 0 && counter_fetch_add_acq_rel(ws_sync + kMaxSyncUnits + sp.c_lo, 1) == sp.n - 1) {
+            arrive[0] = 0;                                    // everyone has passed the wait
+            ws_sync[kMaxSyncUnits + sp.c_lo] = 0;
         }
     }
+    if (nr == 0) return 0;
+    if (!wait_bar(bar, gph & 1, abort_flag, status)) {
+        if (warp == 0) wait_bar_quiet(bar, gph & 1);          // let the copies land
+        return -1;
+    }
+    const float4 *gbuf = reinterpret_cast<const float4 *>(smem + kSmemGather);
+    const float *glse = reinterpret_cast<const float *>(smem + s_lse) + (r_lo - l_lo);
+    float *wsm = reinterpret_cast<float *>(smem + s_w) + warp * sp.n;
+    for (int r = warp; r < nr; r += 4) {
+        float M = -INFINITY;
+        for (int q = lane; q < sp.n; q += 32) M = fmaxf(M, glse[q * nl + r]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int q = lane; q < sp.n; q += 32) {
+            const float l = glse[q * nl + r];
+            const float w = l == -INFINITY ? 0.f : fast_exp2(l - M);   // a partial that saw no key
+            wsm[q] = w;
+            L += w;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        __syncwarp();
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        const float4 *v = gbuf + r * 32 + lane;
+#pragma unroll 4
+        for (int q = 0; q < sp.n; ++q, v += nr * 32) {
+            const float2 w = make_float2(wsm[q], wsm[q]);
+            const float4 x = *v;
+            a0 = ffma2(make_float2(x.x, x.y), w, a0);
+            a1 = ffma2(make_float2(x.z, x.w), w, a1);
+        }
+        __syncwarp();                                         // wsm is rewritten for the next row
+        const int row = r_lo + r;
+        float *dst = out + (((size_t)sp.b * K + row / G) * Hq + sp.g * G + row % G) * kD;
+        reinterpret_cast<float4 *>(dst)[lane] = make_float4(a0.x * inv, a0.y * inv, a1.x * inv, a1.y * inv);
+    }
+    return 1;
 }
 
-__device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, const AttnArgs &p,
-                                              const Decomp &d, int cid, uint32_t tmem)
+__device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem, const AttnArgs &p,
+                                                 const Decomp &d, int cid, uint32_t tmem)
 {
     const int warp = threadIdx.x >> 5;          // 0..3 = TMEM lane quarter
     const int lane = threadIdx.x & 31;
@@ -716,11 +726,16 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
     const int i = m / G;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    const int cs = sh.cs, rank = sh.rank;
 
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
+    if (threadIdx.x == 0) {                      // for the split merge
+        reinterpret_cast<int64_t *>(smem + kSmemPend)[0] = d.W;
+        reinterpret_cast<int *>(smem + kSmemPend)[2] = d.P;
+    }
     Piece pc;
     uint32_t gt = 0, qp = 0, piece = 0, epi = 0;
+    int npend = 0;                               // shared segments awaiting the merge
+    uint32_t gph = 0;                            // B_GATHER phases used
     // all 128 softmax threads meet here; bounded, unlike a named barrier
     auto epi_sync = [&]() -> bool {
         mbar_arrive(sh.bar(B_EPI));
@@ -731,7 +746,7 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
     while (it.next(pc)) {
         const int C = pc.len - p.K;
         const int lim = p.view == ORTHRUS_AR ? C + i : 0x7FFFFFFF;   // last visible key
-        const Tiling tl(pc.a, pc.e, rank, cs);
+        const Tiling tl(pc.a, pc.e);
         float m_run = -INFINITY, l_run = 0.f;
         for (int t = 0; t < tl.ntile; ++t, ++gt) {
             const uint32_t buf = gt % kSBuf;
@@ -811,7 +826,7 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
                     }
                 }
                 const float mb = m_run == -INFINITY ? 0.f : m_run;
-                l_run += softmax_tile(s, nb, sl2, mb, lane_base + buf * 128, __all_sync(0xffffffffu, full));
+                l_run += softmax_tile(s, nb, sl2, mb, lane_base + buf * 128);
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -819,64 +834,104 @@ __device__ __forceinline__ bool softmax_merge(const Shared &sh, uint8_t *smem, c
             if (lane == 0) mbar_arrive(sh.bar(B_PFULL + buf));
         }
 
-        // ---- stage this CTA's (max, sum, O) rows for the owners in the cluster
-        if (tl.ntile > 0) {
+        // ---- write the piece's rows: O normalised by the row sum, staged one
+        // row per thread in the idle K ring (the piece's MMAs are done) and
+        // sent with one bulk copy per row; plus the row's log2-sum-exp when
+        // other CTAs hold the rest of the segment (merged after the last piece)
+        {
             const uint32_t pg = gt - 1, pb = pg % kSBuf;
             if (!wait_bar(sh.bar(B_PVDONE + pb), (pg / kSBuf) & 1, sh.abort_flag, p.status)) return false;
             tc_fence_after();
         }
-        float *stage_o = reinterpret_cast<float *>(smem + kSmemSendO);
-        float2 *stage_ml = reinterpret_cast<float2 *>(smem + kSmemSendML);
-        // (the K ring is idle: the piece's MMAs are done, and every member
-        // finished reading the previous piece's rows before B_PDONE completed)
-        if (tl.ntile > 0 && warp_ok) {
-            float4 *srow = reinterpret_cast<float4 *>(stage_o + m * kStagePitch);
+        const bool sole = pc.a == 0 && pc.e == pc.len;
+        const size_t slot = (size_t)cid + pc.s;
+        if (!sole && npend < 2) {
+            // (only the first and the last piece of a range can be shared;
+            // kept in shared memory, read back after the last piece)
+            if (threadIdx.x == 0) {
+                SharedPiece sp;
+                sp.s0 = pc.s0;
+                sp.b = pc.b;
+                sp.g = pc.g;
+                sp.s = pc.s;
+                sp.len = pc.len;
+                reinterpret_cast<SharedPiece *>(smem + kSmemPend + 16)[npend] = sp;
+            }
+            ++npend;
+        }
+        if (warp_ok) {
+            // a row can see no key of this piece (AR view, piece past C + i):
+            // zero output, zero weight in the merge
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const float2 inv2 = make_float2(inv, inv);
+            float4 *srow = reinterpret_cast<float4 *>(smem + kSmemStage) + m * (kStagePitch / 4);
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t o[32];
                 tmem_ld32(lane_base + kColO + 32 * ch, o);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    srow[8 * ch + c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
-                                                   __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
+                for (int c = 0; c < 8; ++c) {
+                    const float2 x = fmul2(make_float2(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1])), inv2);
+                    const float2 y = fmul2(make_float2(__uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3])), inv2);
+                    srow[8 * ch + c] = make_float4(x.x, x.y, y.x, y.y);
+                }
+            }
+            fence_proxy_async();                  // the row is visible to the bulk copy
+            if (row_ok) {
+                float *dst = sole ? p.out + (((size_t)pc.b * p.K + i) * p.Hq + pc.g * G + m % G) * kD
+                                  : p.ws_o + (slot * rows + m) * kD;
+                bulk_store(dst, sh.base + kSmemStage + m * kStagePitch * 4, kD * 4);
+                bulk_commit();
+                if (!sole) p.ws_lse[slot * lse_pitch(rows) + m] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
             }
         }
-        stage_ml[m] = (tl.ntile > 0 && row_ok && l_run > 0.f) ? make_float2(m_run, l_run)
-                                                              : make_float2(-INFINITY, 0.f);
-        if (tl.ntile > 0) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sh.bar(B_OFREE));      // TMEM O may be overwritten
-            ++qp;
-        }
-        if (!epi_sync()) return false;                        // staging complete
-        // release-ordered remote arrives: every member's staged rows are
-        // visible once B_PREADY completes
-        if (threadIdx.x < cs) mbar_arrive_remote(map_shared(sh.bar(B_PREADY), threadIdx.x));
-        if (!wait_bar_cluster(sh.bar(B_PREADY), piece & 1, sh.abort_flag, p.status)) return false;
-
-        // ---- merge this CTA's rows across the cluster
-        switch (cs) {
-        case 1: pull_merge<1>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
-        case 2: pull_merge<2>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
-        case 4: pull_merge<4>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
-        default: pull_merge<8>(p, stage_o, stage_ml, pc, cid, rank, rows, G); break;
-        }
-        if (!epi_sync()) return false;                        // this CTA's reads are done
-        if (threadIdx.x < cs) mbar_arrive_remote(map_shared(sh.bar(B_PDONE), threadIdx.x));
-        // nobody reads this CTA's staging buffer any more: the K ring may be
-        // refilled (and the CTA may exit)
-        if (!wait_bar_cluster(sh.bar(B_PDONE), piece & 1, sh.abort_flag, p.status)) return false;
-        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.bar(B_OFREE));          // TMEM O may be overwritten
+        ++qp;
+        bulk_wait_read();                                     // the staging row has been read
+        if (!epi_sync()) return false;
+        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // the K ring may be refilled
         ++piece;
+    }
+    bulk_wait_all();                                          // rows written
+    if (npend == 0) return true;
+
+    // ---- split merge: every CTA of a shared segment publishes its partial
+    // (arrive[c_lo] += 1, release), then merges its share of the segment's
+    // rows (split_merge)
+    fence_proxy_async_global();                               // bulk writes before
+    if (!epi_sync()) return false;                            // the release below
+    Decomp ds;                                                // (the split, from shared memory)
+    ds.W = reinterpret_cast<const int64_t *>(smem + kSmemPend)[0];
+    ds.P = reinterpret_cast<const int *>(smem + kSmemPend)[2];
+    auto shared_piece = [&](int k) {
+        const SharedPiece sp = reinterpret_cast<const SharedPiece *>(smem + kSmemPend + 16)[k];
+        SplitInfo si;
+        si.b = sp.b;
+        si.g = sp.g;
+        si.s = sp.s;
+        si.c_lo = cta_of(ds, sp.s0);
+        si.n = cta_of(ds, sp.s0 + sp.len - 1) - si.c_lo + 1;
+        return si;
+    };
+    if (threadIdx.x == 0)
+        for (int k = 0; k < npend; ++k) counter_add_release(p.ws_sync + shared_piece(k).c_lo, 1);
+    for (int k = 0; k < npend; ++k) {
+        if (k > 0 && !epi_sync()) return false;               // gather buffer free again
+        const SplitInfo sp = shared_piece(k);
+        const int used = split_merge(sh.base, sh.abort_flag, smem, p.ws_sync, p.ws_o, p.ws_lse, p.out,
+                                     p.status, sp, cid, rows, G, p.K, p.Hq, gph);
+        if (used < 0) return false;
+        gph += used;
     }
     return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs p, int nclusters)
+                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs p)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -885,12 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Shared sh;
     sh.base = aligned;
     sh.abort_flag = reinterpret_cast<volatile int *>(base_ptr + kSmemMisc + 4);
-    uint32_t cs_u, cid_u;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs_u));
-    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(cid_u));
-    sh.cs = (int)cs_u;
-    sh.rank = (int)cluster_rank();
-    const int cid = (int)cid_u;
+    const int cid = blockIdx.x;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(base_ptr + kSmemMisc);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -914,9 +964,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(sh.bar(B_OFREE), 4);
         mbar_init(sh.bar(B_EPI), 128);
-        mbar_init(sh.bar(B_PREADY), sh.cs);
-        mbar_init(sh.bar(B_PDONE), sh.cs);
         mbar_init(sh.bar(B_MERGED), 1);
+        mbar_init(sh.bar(B_GATHER), 1);
         mbar_init(sh.bar(B_DRAIN), 1);
         *sh.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -934,21 +983,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    // every CTA of the cluster has initialised its barriers before any remote arrive
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
     // ---- everything below may read what earlier kernels wrote
     pdl_wait();
-    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, nclusters, p.min_keys);
+    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, gridDim.x, p.min_keys);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         for (int b = 0; b < p.B; ++b)
             if (seg_len(p.ctx_lens, b, p.K, p.S_max) == 0) raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
     }
-    if (d.W > 0 && cid < d.P) {                  // uniform per cluster
+    if (d.W > 0 && cid < d.P) {
         if (warp < 4) {
-            softmax_merge(sh, base_ptr, p, d, cid, tmem);
+            softmax_epilogue(sh, base_ptr, p, d, cid, tmem);
+            bulk_wait_all();                      // (also after an abort)
         } else if (warp == 4) {
             if (lane == 0) producer(sh, p, d, cid, &tm_q, &tm_k, &tm_v);
             __syncwarp();
@@ -959,13 +1008,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
-    if (*sh.abort_flag && threadIdx.x == 0) {
-        // an aborted cluster member lingers so that peers still reading its
-        // shared memory (or timing out) finish first
-        const unsigned long long t0 = global_ns();
-        while (global_ns() - t0 < 3 * kTimeoutNs) {}
-    }
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -1027,73 +1069,44 @@ bool attn_tc_supported(int dtype, int D, int rows)
 
 namespace {
 
-struct ClusterPlan {
-    int cs = 0;          // CTAs per cluster
-    int nclusters = 0;   // co-resident clusters (the work units of the split)
-};
-
-// Cluster size and count for this device, chosen once: the largest cluster
-// size whose co-resident CTAs cover at least 85% of the SMs (fewer, larger
-// clusters mean fewer split partials), else the size with the most CTAs.
-// ORTHRUS_CLUSTER_SIZE overrides the size (1, 2, 4 or 8).
-ClusterPlan cluster_plan()
+// CTAs of the split for this device, chosen once: one CTA per SM (the
+// kernel's shared memory admits no second one), every CTA resident at once.
+int resident_ctas()
 {
-    static ClusterPlan plans[64];
+    static int ctas[64];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ClusterPlan{};
-    ClusterPlan &pl = plans[dev];
-    if (pl.cs) return pl;
-    int sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (ctas[dev]) return ctas[dev];
+    int sms = 0, per_sm = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::kSmemAlloc) != cudaSuccess)
-        return ClusterPlan{};
-    cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    int forced = 0;
-    if (const char *env = getenv("ORTHRUS_CLUSTER_SIZE")) forced = atoi(env);
-    const int sizes[4] = {8, 4, 2, 1};
-    ClusterPlan best, most;
-    for (int cs : sizes) {
-        if (forced && cs != forced) continue;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(cs * (sms / cs));
-        cfg.blockDim = dim3(tc::kThreads);
-        cfg.dynamicSmemBytes = tc::kSmemAlloc;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = cs;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, tc::attn_tc_kernel, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            continue;
-        }
-        if (n <= 0) continue;
-        if (n * cs > most.nclusters * most.cs) most = ClusterPlan{cs, n};
-        if (!best.cs && n * cs * 100 >= sms * 85) best = ClusterPlan{cs, n};
+                             (int)tc::kSmemAlloc) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::attn_tc_kernel, tc::kThreads,
+                                                      tc::kSmemAlloc) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        return 0;
     }
-    pl = best.cs ? best : most;
-    return pl;
+    // (capped by the split-merge counter block of the workspace)
+    ctas[dev] = sms * per_sm < kMaxSyncUnits ? sms * per_sm : kMaxSyncUnits;
+    return ctas[dev];
 }
 
 }  // namespace
 
 bool attn_tc_plan(int *units, int *min_keys)
 {
-    const ClusterPlan pl = cluster_plan();
-    if (!pl.cs) return false;
-    *units = pl.nclusters;
-    *min_keys = 128 * pl.cs;
+    const int n = resident_ctas();
+    if (!n) return false;
+    *units = n;
+    *min_keys = 128;          // one tile
     return true;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st)
 {
-    const ClusterPlan pl = cluster_plan();
-    if (!pl.cs || units < 1 || units > pl.nclusters) return cudaErrorInvalidValue;
+    const int n = resident_ctas();
+    if (!n || units < 1 || units > n) return cudaErrorInvalidValue;
     const int G = p.Hq / p.Hkv;
     CUtensorMap tq, tk, tv;
     const uint64_t row = tc::kD * 2;
@@ -1104,22 +1117,16 @@ cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st)
                    (uint64_t)p.S_max * row, 64, 64, 1))
         return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.cs * units);
+    cfg.gridDim = dim3(units);
     cfg.blockDim = dim3(tc::kThreads);
     cfg.dynamicSmemBytes = tc::kSmemAlloc;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tk, tv, p, units);
-    if (e != cudaSuccess) return e;
-    return launch_attn_combine(p, units, st);
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tk, tv, p);
 }
 
 }  // namespace orthrus

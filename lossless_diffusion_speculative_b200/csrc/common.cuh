@@ -86,6 +86,7 @@ struct Piece {
     int s;          // segment index b*Hkv + g
     int len;        // segment length (ctx_b + K)
     int a, e;       // key range [a, e) within the segment, 0 <= a < e <= len
+    int64_t s0;     // flat start of the segment
 };
 
 // Iterates the pieces of CTA c in flat order.  Usage:
@@ -137,6 +138,7 @@ struct PieceIter {
             p.len = len_b;
             p.a = (int)a;
             p.e = (int)e;
+            p.s0 = s0;
             ++g;
             if (e > a) return true;
         }

@@ -15,8 +15,9 @@ struct AttnArgs {
     const void *v_cache;
     const int32_t *ctx_lens;
     float *out;
+    int32_t *ws_sync;    // [2, kMaxSyncUnits] split-merge counters (zero between calls)
     float *ws_o;         // [slots, rows, D] split partials (O normalised)
-    float *ws_lse;       // [slots, rows]    log2-sum-exp of each partial
+    float *ws_lse;       // [slots, lse_pitch(rows)] log2-sum-exp of each partial
     int32_t *status;
     int B, Hq, Hkv, D, S_max, K;
     int view;            // orthrus_view
@@ -25,20 +26,26 @@ struct AttnArgs {
     int min_keys;        // smallest key range worth a CTA
 };
 
-// Workspace layout shared by the attention paths: `slots` fp32 partial tiles
-// [rows, D], then their log2-sum-exp values [rows].
-constexpr int kMaxSplitRanks = 8;   // largest cluster the tensor-core path uses
+// Workspace layout shared by the attention paths: a fixed block of counters
+// used by the tensor-core path's in-kernel split merge (arrive[u], depart[u]
+// for the split unit u that opens a segment; zero before and after every
+// call), then `slots` fp32 partial tiles [rows, D], then their log2-sum-exp
+// values [rows].
+constexpr int kMaxSyncUnits = 160;     // >= the tensor-core path's CTA count (148 on B200)
+constexpr size_t kSyncBytes = 2 * kMaxSyncUnits * sizeof(int32_t);
 inline size_t attn_ws_o_bytes(int slots, int rows, int D)
 {
     return ((size_t)slots * rows * D * sizeof(float) + 255) & ~(size_t)255;
 }
+// log2-sum-exp rows are padded to whole 16-byte groups (bulk-copyable)
+__host__ __device__ inline int lse_pitch(int rows) { return (rows + 3) & ~3; }
 inline size_t attn_ws_lse_bytes(int slots, int rows)
 {
-    return ((size_t)slots * rows * sizeof(float) + 255) & ~(size_t)255;
+    return ((size_t)slots * lse_pitch(rows) * sizeof(float) + 255) & ~(size_t)255;
 }
 inline size_t attn_ws_bytes(int slots, int rows, int D)
 {
-    return attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
+    return kSyncBytes + attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);

@@ -163,3 +163,26 @@ def test_repeatable_bitwise():
     a = run_attn(ob.AR, *args, c, torch.bfloat16)
     b = run_attn(ob.AR, *args, c, torch.bfloat16)
     assert torch.equal(a, b)
+
+
+def test_workspace_reused_across_calls_and_shapes():
+    """One workspace, zero-filled once, serves consecutive calls of different
+    context lengths, views and batch shapes: every call matches the oracle and
+    leaves the split-merge counter block (the workspace's first 1280 bytes)
+    zero again."""
+    cases = [(11, 1, [5000]), (12, 2, [3000, 700]), (13, 3, [1, 2500, 129]), (14, 1, [200])]
+    need = max(ob.orthrus_attn_workspace_size(B, 32, 8, 128, 32, torch.bfloat16) for _, B, _ in cases)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for seed, B, lens in cases:
+        q, kc, vc, ctx = _custom(seed, B, 32, 8, 128, 32, lens)
+        for view in (ob.DIFF, ob.AR):
+            out = torch.full((B, 32, 32, 128), float("nan"), dtype=torch.float32, device="cuda")
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            ob.orthrus_attn(view, to_dev(q, torch.bfloat16), to_dev(kc, torch.bfloat16),
+                            to_dev(vc, torch.bfloat16), torch.from_numpy(ctx).cuda(), out, ws,
+                            status=status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            assert int(ws[:1280].count_nonzero().item()) == 0, "split-merge counters left set"
+            assert_attn_close(out.cpu().numpy(), oracle.attention(view, q, kc, vc, ctx),
+                              f"reuse B={B} view={view}")
