@@ -49,18 +49,16 @@ namespace tc {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
-constexpr int kSBuf = 3;
+constexpr int kKStages = 3;                 // K tiles, and each piece's queries
+constexpr int kVStages = 4;
+constexpr int kSBuf = 2;
 constexpr int kThreads = 192;
 constexpr int kBoxKeys = 64;
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B = 16 KiB
-constexpr uint32_t kQBytes = 2 * kHalfBytes;            // 32 KiB
-constexpr uint32_t kStageBytes = 2 * kHalfBytes;        // 128 keys x 256 B
+constexpr uint32_t kStageBytes = 2 * kHalfBytes;        // 128 keys (or query rows) x 256 B
 constexpr uint32_t kBoxBytes = kBoxKeys * 128;          // 8 KiB (64 keys x 64 dims)
 constexpr uint32_t kStagePitch = 132;                  // floats per staged O row (conflict-free)
-constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemK = kSmemQ + kQBytes;
+constexpr uint32_t kSmemK = 0;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 // staging rows for the output bulk copies after a piece, in the K ring (idle
@@ -71,15 +69,14 @@ static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemV, "staging rows fit 
 // split merge, after the last piece, over the idle K and V rings: the
 // gathered partial rows (n x nr rows of D floats, n * nr < rows + n <= 128 +
 // kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
-// one weight row per warp (4 x n floats)
+// two weight rows per warp (8 x n floats)
 constexpr uint32_t kSmemGather = kSmemK;
 static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
-                      4 * kMaxSyncUnits * 4 <= kSmemBar,
+                      8 * kMaxSyncUnits * 4 <= kSmemBar,
               "split merge fits in the rings");
 
 enum : int {
-    B_QFULL = 0,
-    B_QEMPTY,
+    B_QEMPTY = 0,   // the piece's S MMAs are done with Q in TMEM
     B_KFULL,
     B_KEMPTY = B_KFULL + kKStages,
     B_VFULL = B_KEMPTY + kKStages,
@@ -101,7 +98,8 @@ constexpr uint32_t kSmemPend = kSmemMisc + 16;
 constexpr uint32_t kSmemUsed = kSmemPend + 16 + 2 * 32;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = kSBuf * 128;                 // 384
+constexpr uint32_t kColO = kSBuf * 128;                 // 256: O accumulator
+constexpr uint32_t kColQ = kColO + 128;                 // 384: Q, the A operand of S (64 columns)
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -134,6 +132,20 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of a phase (for polling several barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -207,15 +219,11 @@ __device__ __forceinline__ void tc_commit(uint32_t bar)
                  : "memory");
 }
 
-__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t acc)
+// Copy a 128-row x 32-byte slice of a shared-memory matrix (matrix
+// descriptor) into TMEM: row r into lane r, 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
@@ -442,6 +450,9 @@ struct Shared {
 // range (Q loads, MMAs, O use), `kv`/`gt` count tiles.  Every barrier phase
 // is awaited in order.
 
+// The K ring carries, per piece, the piece's queries (one item laid out like a
+// K tile: 2 halves x 128 rows x 128 B, copied into TMEM by the MMA thread)
+// followed by its K tiles; the V ring carries the V tiles.
 __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
                                          int cid, const CUtensorMap *tq, const CUtensorMap *tk,
                                          const CUtensorMap *tv)
@@ -450,60 +461,64 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     const uint32_t q_bytes = 2u * 128u * G * p.K;
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t piece = 0, qp = 0, kv = 0;
+    uint32_t piece = 0, kq = 0, kv = 0;          // K-ring items, V-ring items
     bool ok = true;
+    // next free slot of a ring (false: aborted)
+    auto slot = [&](uint32_t item, int nst, int bfull, int bempty, uint32_t &full, uint32_t &dst,
+                    uint32_t ring) -> bool {
+        const uint32_t st = item % nst, n = item / nst;
+        if (n > 0 && !wait_bar(sh.bar(bempty + st), (n - 1) & 1, sh.abort_flag, p.status)) return false;
+        full = sh.bar(bfull + st);
+        dst = sh.base + ring + st * kStageBytes;
+        return true;
+    };
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
-        // the K and V rings held the previous piece's merge buffers
+        // the K and V rings held the previous piece's output rows
         if (piece > 0 && !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
             ok = false;
             break;
         }
-        if (tl.ntile > 0) {
-            if (qp > 0 && !wait_bar(sh.bar(B_QEMPTY), (qp - 1) & 1, sh.abort_flag, p.status)) {
-                ok = false;
-                break;
-            }
-            mbar_expect_tx(sh.bar(B_QFULL), q_bytes);
-            tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, pc.b * p.K);
-            tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, pc.b * p.K);
+        uint32_t full, dst;
+        if (!slot(kq, kKStages, B_KFULL, B_KEMPTY, full, dst, kSmemK)) {
+            ok = false;
+            break;
         }
+        mbar_expect_tx(full, q_bytes);
+        tma_load_3d(dst, tq, full, 0, pc.g * G, pc.b * p.K);
+        tma_load_3d(dst + kHalfBytes, tq, full, 64, pc.g * G, pc.b * p.K);
+        ++kq;
         const int z = pc.b * p.Hkv + pc.g;
-        for (int t = 0; t < tl.ntile && ok; ++t, ++kv) {
+        for (int t = 0; t < tl.ntile && ok; ++t) {
             const int nb = tl.boxes_in_tile(t);
             for (int which = 0; which < 2; ++which) {
-                const uint32_t nst = which ? kVStages : kKStages;
-                const uint32_t st = kv % nst, n = kv / nst;
-                const uint32_t full = sh.bar((which ? B_VFULL : B_KFULL) + st);
-                const uint32_t empty = sh.bar((which ? B_VEMPTY : B_KEMPTY) + st);
-                if (n > 0 && !wait_bar(empty, (n - 1) & 1, sh.abort_flag, p.status)) {
+                if (!(which ? slot(kv, kVStages, B_VFULL, B_VEMPTY, full, dst, kSmemV)
+                            : slot(kq, kKStages, B_KFULL, B_KEMPTY, full, dst, kSmemK))) {
                     ok = false;
                     break;
                 }
                 mbar_expect_tx(full, nb * 2u * kBoxBytes);
-                const uint32_t dst = sh.base + (which ? kSmemV : kSmemK) + st * kStageBytes;
                 const CUtensorMap *m = which ? tv : tk;
                 for (int kb = 0; kb < nb; ++kb) {
                     const int y = tl.box_start(tl.box_of(t, kb));
                     tma_load_3d(dst + kb * kBoxBytes, m, full, 0, y, z);
                     tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, m, full, 64, y, z);
                 }
+                ++(which ? kv : kq);
             }
         }
-        if (tl.ntile > 0) ++qp;
         ++piece;
     }
     if (!ok) {
         // abort: let every copy already issued land before the CTA exits
         for (uint32_t s = 0; s < kKStages; ++s) {
-            const uint32_t fills = kv / kKStages + (s < kv % kKStages ? 1u : 0u);
+            const uint32_t fills = kq / kKStages + (s < kq % kKStages ? 1u : 0u);
             if (fills) wait_bar_quiet(sh.bar(B_KFULL + s), (fills - 1) & 1);
         }
         for (uint32_t s = 0; s < kVStages; ++s) {
             const uint32_t fills = kv / kVStages + (s < kv % kVStages ? 1u : 0u);
             if (fills) wait_bar_quiet(sh.bar(B_VFULL + s), (fills - 1) & 1);
         }
-        if (qp > 0) wait_bar_quiet(sh.bar(B_QFULL), (qp - 1) & 1);
     }
 }
 
@@ -513,67 +528,95 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     const uint32_t idesc_pv = instr_desc(128, 128, true);
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t qp = 0, kv = 0, gt = 0;
+    uint32_t qp = 0, kq = 0, kv = 0, gt = 0;     // pieces, K-ring items, V tiles, tiles
     bool ok = true;
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
-        if (tl.ntile == 0) continue;
-        if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        for (int t = 0; t <= tl.ntile && ok; ++t) {
-            if (t < tl.ntile) {        // S(t) = Q K(t)^T
-                const int nb = tl.boxes_in_tile(t);
-                const uint32_t st = (kv + t) % kKStages, n = (kv + t) / kKStages;
-                const uint32_t g = gt + t, buf = g % kSBuf;
-                if (!wait_bar(sh.bar(B_KFULL + st), n & 1, sh.abort_flag, p.status)) { ok = false; break; }
-                if (g >= kSBuf &&
-                    !wait_bar(sh.bar(B_PVDONE + buf), (g / kSBuf - 1) & 1, sh.abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t idesc_s = instr_desc(128, 64 * nb, false);
-                const uint32_t kaddr = sh.base + kSmemK + st * kStageBytes;
-                const uint32_t qaddr = sh.base + kSmemQ;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    tc_mma_ss(tmem + buf * 128, smem_desc(qaddr + off, 16, 1024),
-                              smem_desc(kaddr + off, 16, 1024), idesc_s, kk > 0);
-                }
-                tc_commit(sh.bar(B_SFULL + buf));
-                tc_commit(sh.bar(B_KEMPTY + st));
-                if (t == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
+        {   // the piece's queries: K-ring item -> TMEM columns [kColQ, kColQ + 64)
+            const uint32_t st = kq % kKStages, n = kq / kKStages;
+            if (!wait_bar(sh.bar(B_KFULL + st), n & 1, sh.abort_flag, p.status) ||
+                (qp > 0 && !wait_bar(sh.bar(B_QEMPTY), (qp - 1) & 1, sh.abort_flag, p.status))) {
+                ok = false;
+                break;
             }
-            if (t >= 1) {              // O += P(t-1) V(t-1)
-                const int tp = t - 1;
-                const int nb = tl.boxes_in_tile(tp);
-                const uint32_t st = (kv + tp) % kVStages, n = (kv + tp) / kVStages;
-                const uint32_t g = gt + tp, buf = g % kSBuf;
-                if (!wait_bar(sh.bar(B_PFULL + buf), (g / kSBuf) & 1, sh.abort_flag, p.status) ||
-                    !wait_bar(sh.bar(B_VFULL + st), n & 1, sh.abort_flag, p.status)) {
-                    ok = false;
-                    break;
+            tc_fence_after();
+            const uint32_t qaddr = sh.base + kSmemK + st * kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)      // 16 head dims per slice
+                tc_cp_128x256b(tmem + kColQ + 8 * kk,
+                               smem_desc(qaddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024));
+            tc_commit(sh.bar(B_KEMPTY + st));    // the slot is free once copied
+            ++kq;
+        }
+        // S(t) and PV(t) are issued as soon as their inputs are ready (S first
+        // when both are: it feeds the softmax), so a late K tile does not hold
+        // back the PV of the tile before it
+        int ns = 0, npv = 0;
+        unsigned long long t0 = 0;
+        uint32_t idle = 0;
+        while (npv < tl.ntile) {
+            bool issued = false;
+            if (ns < tl.ntile) {       // S(ns) = Q K(ns)^T
+                const uint32_t st = (kq + ns) % kKStages, n = (kq + ns) / kKStages;
+                const uint32_t g = gt + ns, buf = g % kSBuf;
+                if (mbar_test(sh.bar(B_KFULL + st), n & 1) &&
+                    (g < kSBuf || mbar_test(sh.bar(B_PVDONE + buf), (g / kSBuf - 1) & 1))) {
+                    tc_fence_after();
+                    const int nb = tl.boxes_in_tile(ns);
+                    const uint32_t idesc_s = instr_desc(128, 64 * nb, false);
+                    const uint32_t kaddr = sh.base + kSmemK + st * kStageBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {   // 16 head dims per step; A = Q in TMEM
+                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                        tc_mma_ts(tmem + buf * 128, tmem + kColQ + 8 * kk, smem_desc(kaddr + off, 16, 1024),
+                                  idesc_s, kk > 0);
+                    }
+                    tc_commit(sh.bar(B_SFULL + buf));
+                    tc_commit(sh.bar(B_KEMPTY + st));
+                    if (ns == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
+                    ++ns;
+                    issued = true;
                 }
-                if (tp == 0 && qp > 0 &&
-                    !wait_bar(sh.bar(B_OFREE), (qp - 1) & 1, sh.abort_flag, p.status)) {
-                    ok = false;
-                    break;
+            }
+            if (!issued && npv < ns) {   // O += P(npv) V(npv)
+                const uint32_t st = (kv + npv) % kVStages, n = (kv + npv) / kVStages;
+                const uint32_t g = gt + npv, buf = g % kSBuf;
+                if (mbar_test(sh.bar(B_PFULL + buf), (g / kSBuf) & 1) && mbar_test(sh.bar(B_VFULL + st), n & 1) &&
+                    (npv > 0 || qp == 0 || mbar_test(sh.bar(B_OFREE), (qp - 1) & 1))) {
+                    tc_fence_after();
+                    const int nb = tl.boxes_in_tile(npv);
+                    const uint32_t vaddr = sh.base + kSmemV + st * kStageBytes;
+                    const int steps = 4 * nb;
+                    for (int kk = 0; kk < steps; ++kk)
+                        tc_mma_ts(tmem + kColO, tmem + buf * 128 + 8 * kk,
+                                  smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                                  (npv == 0 && kk == 0) ? 0u : 1u);
+                    for (int kk = 0; kk < steps; ++kk)
+                        tc_mma_ts(tmem + kColO, tmem + buf * 128 + 64 + 8 * kk,
+                                  smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
+                    tc_commit(sh.bar(B_VEMPTY + st));
+                    tc_commit(sh.bar(B_PVDONE + buf));
+                    ++npv;
+                    issued = true;
                 }
-                tc_fence_after();
-                const uint32_t vaddr = sh.base + kSmemV + st * kStageBytes;
-                const int steps = 4 * nb;
-                for (int kk = 0; kk < steps; ++kk)
-                    tc_mma_ts(tmem + kColO, tmem + buf * 128 + 8 * kk,
-                              smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                              (tp == 0 && kk == 0) ? 0u : 1u);
-                for (int kk = 0; kk < steps; ++kk)
-                    tc_mma_ts(tmem + kColO, tmem + buf * 128 + 64 + 8 * kk,
-                              smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
-                tc_commit(sh.bar(B_VEMPTY + st));
-                tc_commit(sh.bar(B_PVDONE + buf));
+            }
+            if (issued) {
+                idle = 0;
+            } else {                    // bounded: the same limit as wait_bar
+                if (idle == 0) t0 = global_ns();
+                if ((++idle & 63u) == 0) {
+                    if (*sh.abort_flag) { ok = false; break; }
+                    if (global_ns() - t0 > kTimeoutNs) {
+                        *sh.abort_flag = 1;
+                        raise_status(p.status, ORTHRUS_STATUS_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                }
+                __nanosleep(20);
             }
         }
+        kq += tl.ntile;
         kv += tl.ntile;
         gt += tl.ntile;
         ++qp;
@@ -623,9 +666,9 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
 // of the rows of all n partials, with their log2-sum-exp values, into shared
 // memory (lane q issues the bulk copies of partial q), and thread 0 leaves
 // (depart[c_lo] += 1; the last to leave resets both counters).  Each warp then
-// merges whole rows: lanes compute the weights 2^(lse_q - max) / sum of the
-// row's partials (the log-sum-exp merge of flash-decoding), then lane c4
-// accumulates 16-byte column c4 over the partials and stores it.
+// merges whole rows, two at a time: lanes compute the weights 2^(lse_q - max)
+// / sum of the rows' partials (the log-sum-exp merge of flash-decoding), then
+// lane c4 accumulates 16-byte column c4 over the partials and stores it.
 // Returns the B_GATHER phases used (0 or 1), or -1 after an abort.
 __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag, uint8_t *smem,
                                         int32_t *ws_sync, const float *ws_o, const float *ws_lse,
@@ -640,7 +683,7 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
     const int l_lo = r_lo & ~3, nl = ((r_lo + nr + 3) & ~3) - l_lo;   // 16-byte lse rows
     const uint32_t o_bytes = (uint32_t)nr * kD * 4, l_bytes = (uint32_t)nl * 4;
     const uint32_t s_lse = kSmemGather + (uint32_t)sp.n * o_bytes;     // after the O rows
-    const uint32_t s_w = s_lse + (((uint32_t)sp.n * l_bytes + 15u) & ~15u);   // [4 warps][n] weights
+    const uint32_t s_w = s_lse + (((uint32_t)sp.n * l_bytes + 15u) & ~15u);   // [4 warps][2][n] weights
     int32_t *arrive = ws_sync + sp.c_lo;
     if (warp == 0) {
         bool ok = true;
@@ -679,36 +722,58 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
     }
     const float4 *gbuf = reinterpret_cast<const float4 *>(smem + kSmemGather);
     const float *glse = reinterpret_cast<const float *>(smem + s_lse) + (r_lo - l_lo);
-    float *wsm = reinterpret_cast<float *>(smem + s_w) + warp * sp.n;
-    for (int r = warp; r < nr; r += 4) {
-        float M = -INFINITY;
-        for (int q = lane; q < sp.n; q += 32) M = fmaxf(M, glse[q * nl + r]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
+    float *wsm = reinterpret_cast<float *>(smem + s_w) + warp * 2 * sp.n;
+    // each warp merges rows r and r + 4 together (two independent chains)
+    for (int r = warp; r < nr; r += 8) {
+        const int r1 = r + 4 < nr ? r + 4 : r;              // (a repeat is not stored)
+        float M0 = -INFINITY, M1 = -INFINITY;
         for (int q = lane; q < sp.n; q += 32) {
-            const float l = glse[q * nl + r];
-            const float w = l == -INFINITY ? 0.f : fast_exp2(l - M);   // a partial that saw no key
-            wsm[q] = w;
-            L += w;
+            M0 = fmaxf(M0, glse[q * nl + r]);
+            M1 = fmaxf(M1, glse[q * nl + r1]);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        for (int o = 16; o > 0; o >>= 1) {
+            M0 = fmaxf(M0, __shfl_xor_sync(0xffffffffu, M0, o));
+            M1 = fmaxf(M1, __shfl_xor_sync(0xffffffffu, M1, o));
+        }
+        float L0 = 0.f, L1 = 0.f;
+        for (int q = lane; q < sp.n; q += 32) {
+            const float l0 = glse[q * nl + r], l1 = glse[q * nl + r1];
+            const float w0 = l0 == -INFINITY ? 0.f : fast_exp2(l0 - M0);   // a partial that
+            const float w1 = l1 == -INFINITY ? 0.f : fast_exp2(l1 - M1);   // saw no key
+            wsm[q] = w0;
+            wsm[sp.n + q] = w1;
+            L0 += w0;
+            L1 += w1;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            L0 += __shfl_xor_sync(0xffffffffu, L0, o);
+            L1 += __shfl_xor_sync(0xffffffffu, L1, o);
+        }
         __syncwarp();
-        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
         float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-        const float4 *v = gbuf + r * 32 + lane;
-#pragma unroll 4
-        for (int q = 0; q < sp.n; ++q, v += nr * 32) {
-            const float2 w = make_float2(wsm[q], wsm[q]);
-            const float4 x = *v;
+        float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
+        const float4 *v = gbuf + r * 32 + lane, *u = gbuf + r1 * 32 + lane;
+#pragma unroll 2
+        for (int q = 0; q < sp.n; ++q, v += nr * 32, u += nr * 32) {
+            const float2 w = make_float2(wsm[q], wsm[q]), z = make_float2(wsm[sp.n + q], wsm[sp.n + q]);
+            const float4 x = *v, y = *u;
             a0 = ffma2(make_float2(x.x, x.y), w, a0);
             a1 = ffma2(make_float2(x.z, x.w), w, a1);
+            b0 = ffma2(make_float2(y.x, y.y), z, b0);
+            b1 = ffma2(make_float2(y.z, y.w), z, b1);
         }
-        __syncwarp();                                         // wsm is rewritten for the next row
-        const int row = r_lo + r;
+        __syncwarp();                                         // wsm is rewritten next
+        int row = r_lo + r;
         float *dst = out + (((size_t)sp.b * K + row / G) * Hq + sp.g * G + row % G) * kD;
-        reinterpret_cast<float4 *>(dst)[lane] = make_float4(a0.x * inv, a0.y * inv, a1.x * inv, a1.y * inv);
+        reinterpret_cast<float4 *>(dst)[lane] = make_float4(a0.x * inv0, a0.y * inv0, a1.x * inv0, a1.y * inv0);
+        if (r1 != r) {
+            row = r_lo + r1;
+            dst = out + (((size_t)sp.b * K + row / G) * Hq + sp.g * G + row % G) * kD;
+            reinterpret_cast<float4 *>(dst)[lane] = make_float4(b0.x * inv1, b0.y * inv1, b1.x * inv1, b1.y * inv1);
+        }
     }
     return 1;
 }
@@ -947,7 +1012,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- prologue: touches nothing an earlier kernel in the stream may write
     pdl_trigger();
     if (threadIdx.x == 0) {
-        mbar_init(sh.bar(B_QFULL), 1);
         mbar_init(sh.bar(B_QEMPTY), 1);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(sh.bar(B_KFULL + s), 1);
