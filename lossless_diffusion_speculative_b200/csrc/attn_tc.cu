@@ -452,7 +452,9 @@ struct Shared {
 
 // The K ring carries, per piece, the piece's queries (one item laid out like a
 // K tile: 2 halves x 128 rows x 128 B, copied into TMEM by the MMA thread)
-// followed by its K tiles; the V ring carries the V tiles.
+// followed by its K tiles; the V ring carries the V tiles.  Each ring is filled
+// as soon as it has a free slot (K before V when both have), so a V tile never
+// waits for a K slot or the other way round.
 __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
                                          int cid, const CUtensorMap *tq, const CUtensorMap *tk,
                                          const CUtensorMap *tv)
@@ -463,14 +465,9 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     Piece pc;
     uint32_t piece = 0, kq = 0, kv = 0;          // K-ring items, V-ring items
     bool ok = true;
-    // next free slot of a ring (false: aborted)
-    auto slot = [&](uint32_t item, int nst, int bfull, int bempty, uint32_t &full, uint32_t &dst,
-                    uint32_t ring) -> bool {
-        const uint32_t st = item % nst, n = item / nst;
-        if (n > 0 && !wait_bar(sh.bar(bempty + st), (n - 1) & 1, sh.abort_flag, p.status)) return false;
-        full = sh.bar(bfull + st);
-        dst = sh.base + ring + st * kStageBytes;
-        return true;
+    auto slot_free = [&](uint32_t item, int nst, int bempty) {
+        const uint32_t n = item / nst;
+        return n == 0 || mbar_test(sh.bar(bempty + item % nst), (n - 1) & 1);
     };
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
@@ -479,32 +476,63 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
             ok = false;
             break;
         }
-        uint32_t full, dst;
-        if (!slot(kq, kKStages, B_KFULL, B_KEMPTY, full, dst, kSmemK)) {
-            ok = false;
-            break;
-        }
-        mbar_expect_tx(full, q_bytes);
-        tma_load_3d(dst, tq, full, 0, pc.g * G, pc.b * p.K);
-        tma_load_3d(dst + kHalfBytes, tq, full, 64, pc.g * G, pc.b * p.K);
-        ++kq;
         const int z = pc.b * p.Hkv + pc.g;
-        for (int t = 0; t < tl.ntile && ok; ++t) {
-            const int nb = tl.boxes_in_tile(t);
-            for (int which = 0; which < 2; ++which) {
-                if (!(which ? slot(kv, kVStages, B_VFULL, B_VEMPTY, full, dst, kSmemV)
-                            : slot(kq, kKStages, B_KFULL, B_KEMPTY, full, dst, kSmemK))) {
-                    ok = false;
-                    break;
+        int nk = 0, nv = 0;                      // this piece's items: K ring (queries first), V ring
+        unsigned long long t0 = 0;
+        uint32_t idle = 0;
+        while (nk <= tl.ntile || nv < tl.ntile) {
+            bool issued = false;
+            for (int pass = 0; pass < 2 && !issued; ++pass) {
+                // K first unless the K stream is ahead of the V stream
+                const bool use_k = (pass == 0) == (nk - 1 <= nv);
+                if (use_k && nk <= tl.ntile && slot_free(kq, kKStages, B_KEMPTY)) {
+                    const uint32_t full = sh.bar(B_KFULL + kq % kKStages);
+                    const uint32_t dst = sh.base + kSmemK + (kq % kKStages) * kStageBytes;
+                    if (nk == 0) {
+                        mbar_expect_tx(full, q_bytes);
+                        tma_load_3d(dst, tq, full, 0, pc.g * G, pc.b * p.K);
+                        tma_load_3d(dst + kHalfBytes, tq, full, 64, pc.g * G, pc.b * p.K);
+                    } else {
+                        const int t = nk - 1, nb = tl.boxes_in_tile(t);
+                        mbar_expect_tx(full, nb * 2u * kBoxBytes);
+                        for (int kb = 0; kb < nb; ++kb) {
+                            const int y = tl.box_start(tl.box_of(t, kb));
+                            tma_load_3d(dst + kb * kBoxBytes, tk, full, 0, y, z);
+                            tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, tk, full, 64, y, z);
+                        }
+                    }
+                    ++nk;
+                    ++kq;
+                    issued = true;
+                } else if (!use_k && nv < tl.ntile && slot_free(kv, kVStages, B_VEMPTY)) {
+                    const uint32_t full = sh.bar(B_VFULL + kv % kVStages);
+                    const uint32_t dst = sh.base + kSmemV + (kv % kVStages) * kStageBytes;
+                    const int t = nv, nb = tl.boxes_in_tile(t);
+                    mbar_expect_tx(full, nb * 2u * kBoxBytes);
+                    for (int kb = 0; kb < nb; ++kb) {
+                        const int y = tl.box_start(tl.box_of(t, kb));
+                        tma_load_3d(dst + kb * kBoxBytes, tv, full, 0, y, z);
+                        tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, tv, full, 64, y, z);
+                    }
+                    ++nv;
+                    ++kv;
+                    issued = true;
                 }
-                mbar_expect_tx(full, nb * 2u * kBoxBytes);
-                const CUtensorMap *m = which ? tv : tk;
-                for (int kb = 0; kb < nb; ++kb) {
-                    const int y = tl.box_start(tl.box_of(t, kb));
-                    tma_load_3d(dst + kb * kBoxBytes, m, full, 0, y, z);
-                    tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, m, full, 64, y, z);
+            }
+            if (issued) {
+                idle = 0;
+            } else {                    // bounded: the same limit as wait_bar
+                if (idle == 0) t0 = global_ns();
+                if ((++idle & 63u) == 0) {
+                    if (*sh.abort_flag) { ok = false; break; }
+                    if (global_ns() - t0 > kTimeoutNs) {
+                        *sh.abort_flag = 1;
+                        raise_status(p.status, ORTHRUS_STATUS_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
                 }
-                ++(which ? kv : kq);
+                __nanosleep(20);
             }
         }
         ++piece;
