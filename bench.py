@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one attn_tc_kernel launch on the headline workload, from the
 # ncu capture summarised in profiles/ (bytes read + written), keyed by the hash
 # of the kernel source it was taken on; reported as null once the source changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {("qwen3_8b_step", "ac2d6c5915d57c6f"): 37.11e6}
 
 
 def parse():
@@ -354,8 +354,9 @@ def main():
     per_call_s = attn_ms / 1e3 / (2 * st.L)
     achieved = st.kv_bytes_per_attn_call() / per_call_s / 1e9
     traffic = NCU_TRAFFIC.get((w.name, kernel_hash()))
-    launches_per_step = (2 + 2 * st.L * 2 + 2 + 1) if args.order == "cold" else \
-        (2 * st.L + 2 * st.L * 2 + 2 + 1)
+    per_call = 1 if st.tc_path else 2             # tcgen05: one launch; CUDA-core: + combine
+    launches_per_step = (2 + 2 * st.L * per_call + 2 + 1) if args.order == "cold" else \
+        (2 * st.L + 2 * st.L * per_call + 2 + 1)
 
     if rank == 0:
         line = {
@@ -373,7 +374,8 @@ def main():
             "attn_path": "tcgen05" if st.tc_path else "cuda-core",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
-                         "kernel": "orthrus_attn (attn_tc_kernel + attn_combine_kernel)",
+                         "kernel": ("orthrus_attn (attn_tc_kernel, split merge in-kernel)" if st.tc_path
+                                    else "orthrus_attn (attn_simt_kernel + attn_combine_kernel)"),
                          "peak_source": f"{hbm_src} hbm_gbs",
                          "bytes_per_launch": st.kv_bytes_per_attn_call()},
             "gpu_launches": launches_per_step * args.steps,
