@@ -49,8 +49,8 @@ namespace tc {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kKStages = 3;                 // K tiles, and each piece's queries
-constexpr int kVStages = 4;
+constexpr int kKStages = 2;                 // K tiles, and each piece's queries
+constexpr int kVStages = 5;
 constexpr int kSBuf = 2;
 constexpr int kThreads = 192;
 constexpr int kBoxKeys = 64;
@@ -61,11 +61,12 @@ constexpr uint32_t kStagePitch = 132;                  // floats per staged O ro
 constexpr uint32_t kSmemK = 0;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
-// staging rows for the output bulk copies after a piece, in the K ring (idle
-// once the piece's last S MMA has finished); the padded pitch keeps the
-// row-per-thread writes free of bank conflicts
+// staging rows for the output bulk copies after a piece, over the rings (idle
+// once the piece's last PV has finished; the producer starts the next piece
+// only after B_MERGED); the padded pitch keeps the row-per-thread writes free
+// of bank conflicts
 constexpr uint32_t kSmemStage = kSmemK;
-static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemV, "staging rows fit in the K ring");
+static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemBar, "staging rows fit in the rings");
 // split merge, after the last piece, over the idle K and V rings: the
 // gathered partial rows (n x nr rows of D floats, n * nr < rows + n <= 128 +
 // kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
@@ -86,7 +87,7 @@ enum : int {
     B_PVDONE = B_PFULL + kSBuf,
     B_OFREE = B_PVDONE + kSBuf,
     B_EPI,          // the 128 softmax threads (local, bounded)
-    B_MERGED,       // the piece's rows are out: the K ring may be refilled
+    B_MERGED,       // the piece's rows are out: the rings may be refilled
     B_GATHER,       // tx: the split partials of a segment have landed in smem
     B_DRAIN,
     B_COUNT
@@ -592,13 +593,14 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
                     tc_fence_after();
                     const int nb = tl.boxes_in_tile(ns);
                     const uint32_t idesc_s = instr_desc(128, 64 * nb, false);
-                    const uint32_t kaddr = sh.base + kSmemK + st * kStageBytes;
+                    // one descriptor per tile; a step's is this one plus its byte
+                    // offset / 16 (the 14-bit address field cannot carry out)
+                    const uint64_t kd = smem_desc(sh.base + kSmemK + st * kStageBytes, 16, 1024);
+                    const uint32_t dcol = tmem + buf * 128;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {   // 16 head dims per step; A = Q in TMEM
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        tc_mma_ts(tmem + buf * 128, tmem + kColQ + 8 * kk, smem_desc(kaddr + off, 16, 1024),
+                    for (int kk = 0; kk < 8; ++kk)     // 16 head dims per step; A = Q in TMEM
+                        tc_mma_ts(dcol, tmem + kColQ + 8 * kk, kd + (((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4),
                                   idesc_s, kk > 0);
-                    }
                     tc_commit(sh.bar(B_SFULL + buf));
                     tc_commit(sh.bar(B_KEMPTY + st));
                     if (ns == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
@@ -612,16 +614,27 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
                 if (mbar_test(sh.bar(B_PFULL + buf), (g / kSBuf) & 1) && mbar_test(sh.bar(B_VFULL + st), n & 1) &&
                     (npv > 0 || qp == 0 || mbar_test(sh.bar(B_OFREE), (qp - 1) & 1))) {
                     tc_fence_after();
-                    const int nb = tl.boxes_in_tile(npv);
-                    const uint32_t vaddr = sh.base + kSmemV + st * kStageBytes;
-                    const int steps = 4 * nb;
-                    for (int kk = 0; kk < steps; ++kk)
-                        tc_mma_ts(tmem + kColO, tmem + buf * 128 + 8 * kk,
-                                  smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                                  (npv == 0 && kk == 0) ? 0u : 1u);
-                    for (int kk = 0; kk < steps; ++kk)
-                        tc_mma_ts(tmem + kColO, tmem + buf * 128 + 64 + 8 * kk,
-                                  smem_desc(vaddr + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
+                    // 16 keys per step (+2048 B of V, +8 columns of P); the issue
+                    // loops are unrolled with incremented descriptors so that the
+                    // single issuing thread keeps up with the tensor pipe
+                    const uint64_t vd = smem_desc(sh.base + kSmemV + st * kStageBytes, kHalfBytes, 1024);
+                    const uint32_t pcol = tmem + buf * 128, ocol = tmem + kColO;
+                    const uint32_t acc0 = npv == 0 ? 0u : 1u;
+                    if (tl.boxes_in_tile(npv) == 2) {
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
+                    }
                     tc_commit(sh.bar(B_VEMPTY + st));
                     tc_commit(sh.bar(B_PVDONE + buf));
                     ++npv;
@@ -985,7 +998,7 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
         ++qp;
         bulk_wait_read();                                     // the staging row has been read
         if (!epi_sync()) return false;
-        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // the K ring may be refilled
+        if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // the rings may be refilled
         ++piece;
     }
     bulk_wait_all();                                          // rows written
