@@ -49,16 +49,18 @@ namespace tc {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kKStages = 2;                 // K tiles, and each piece's queries
-constexpr int kVStages = 5;
-constexpr int kSBuf = 2;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr int kSBuf = 3;                    // S can run two tiles ahead of PV
 constexpr int kThreads = 192;
 constexpr int kBoxKeys = 64;
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B = 16 KiB
-constexpr uint32_t kStageBytes = 2 * kHalfBytes;        // 128 keys (or query rows) x 256 B
+constexpr uint32_t kQBytes = 2 * kHalfBytes;            // 128 query rows x 256 B
+constexpr uint32_t kStageBytes = 2 * kHalfBytes;        // 128 keys x 256 B
 constexpr uint32_t kBoxBytes = kBoxKeys * 128;          // 8 KiB (64 keys x 64 dims)
 constexpr uint32_t kStagePitch = 132;                  // floats per staged O row (conflict-free)
-constexpr uint32_t kSmemK = 0;
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kSmemQ + kQBytes;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 // staging rows for the output bulk copies after a piece, over the rings (idle
@@ -67,17 +69,18 @@ constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 // of bank conflicts
 constexpr uint32_t kSmemStage = kSmemK;
 static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemBar, "staging rows fit in the rings");
-// split merge, after the last piece, over the idle K and V rings: the
+// split merge, after the last piece, over the idle query tile and rings: the
 // gathered partial rows (n x nr rows of D floats, n * nr < rows + n <= 128 +
 // kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
 // two weight rows per warp (8 x n floats)
-constexpr uint32_t kSmemGather = kSmemK;
+constexpr uint32_t kSmemGather = kSmemQ;
 static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
                       8 * kMaxSyncUnits * 4 <= kSmemBar,
               "split merge fits in the rings");
 
 enum : int {
-    B_QEMPTY = 0,   // the piece's S MMAs are done with Q in TMEM
+    B_QFULL = 0,    // tx: the piece's query tile has landed
+    B_QEMPTY,       // the piece's S MMAs are done with it
     B_KFULL,
     B_KEMPTY = B_KFULL + kKStages,
     B_VFULL = B_KEMPTY + kKStages,
@@ -99,8 +102,7 @@ constexpr uint32_t kSmemPend = kSmemMisc + 16;
 constexpr uint32_t kSmemUsed = kSmemPend + 16 + 2 * 32;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = kSBuf * 128;                 // 256: O accumulator
-constexpr uint32_t kColQ = kColO + 128;                 // 384: Q, the A operand of S (64 columns)
+constexpr uint32_t kColO = kSBuf * 128;                 // 384: O accumulator
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -220,11 +222,15 @@ __device__ __forceinline__ void tc_commit(uint32_t bar)
                  : "memory");
 }
 
-// Copy a 128-row x 32-byte slice of a shared-memory matrix (matrix
-// descriptor) into TMEM: row r into lane r, 8 consecutive 32-bit columns.
-__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc)
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
@@ -451,11 +457,11 @@ struct Shared {
 // range (Q loads, MMAs, O use), `kv`/`gt` count tiles.  Every barrier phase
 // is awaited in order.
 
-// The K ring carries, per piece, the piece's queries (one item laid out like a
-// K tile: 2 halves x 128 rows x 128 B, copied into TMEM by the MMA thread)
-// followed by its K tiles; the V ring carries the V tiles.  Each ring is filled
-// as soon as it has a free slot (K before V when both have), so a V tile never
-// waits for a K slot or the other way round.
+// Per piece: the query tile (2 halves x 128 rows x 128 B, once the previous
+// piece's S MMAs are done with it), then the K tiles into the K ring and the V
+// tiles into the V ring.  Each ring is filled as soon as it has a free slot (K
+// before V when both have), so a V tile never waits for a K slot or the other
+// way round.
 __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
                                          int cid, const CUtensorMap *tq, const CUtensorMap *tk,
                                          const CUtensorMap *tv)
@@ -464,7 +470,7 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     const uint32_t q_bytes = 2u * 128u * G * p.K;
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t piece = 0, kq = 0, kv = 0;          // K-ring items, V-ring items
+    uint32_t piece = 0, qloads = 0, kq = 0, kv = 0;   // pieces, Q tiles, K tiles, V tiles
     bool ok = true;
     auto slot_free = [&](uint32_t item, int nst, int bempty) {
         const uint32_t n = item / nst;
@@ -472,35 +478,37 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     };
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
+        if (piece > 0 && !wait_bar(sh.bar(B_QEMPTY), (piece - 1) & 1, sh.abort_flag, p.status)) {
+            ok = false;
+            break;
+        }
+        mbar_expect_tx(sh.bar(B_QFULL), q_bytes);
+        tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, pc.b * p.K);
+        tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, pc.b * p.K);
+        ++qloads;
         // the K and V rings held the previous piece's output rows
         if (piece > 0 && !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
             ok = false;
             break;
         }
         const int z = pc.b * p.Hkv + pc.g;
-        int nk = 0, nv = 0;                      // this piece's items: K ring (queries first), V ring
+        int nk = 0, nv = 0;                      // this piece's K and V tiles issued
         unsigned long long t0 = 0;
         uint32_t idle = 0;
-        while (nk <= tl.ntile || nv < tl.ntile) {
+        while (nk < tl.ntile || nv < tl.ntile) {
             bool issued = false;
             for (int pass = 0; pass < 2 && !issued; ++pass) {
                 // K first unless the K stream is ahead of the V stream
-                const bool use_k = (pass == 0) == (nk - 1 <= nv);
-                if (use_k && nk <= tl.ntile && slot_free(kq, kKStages, B_KEMPTY)) {
+                const bool use_k = (pass == 0) == (nk <= nv);
+                if (use_k && nk < tl.ntile && slot_free(kq, kKStages, B_KEMPTY)) {
                     const uint32_t full = sh.bar(B_KFULL + kq % kKStages);
                     const uint32_t dst = sh.base + kSmemK + (kq % kKStages) * kStageBytes;
-                    if (nk == 0) {
-                        mbar_expect_tx(full, q_bytes);
-                        tma_load_3d(dst, tq, full, 0, pc.g * G, pc.b * p.K);
-                        tma_load_3d(dst + kHalfBytes, tq, full, 64, pc.g * G, pc.b * p.K);
-                    } else {
-                        const int t = nk - 1, nb = tl.boxes_in_tile(t);
-                        mbar_expect_tx(full, nb * 2u * kBoxBytes);
-                        for (int kb = 0; kb < nb; ++kb) {
-                            const int y = tl.box_start(tl.box_of(t, kb));
-                            tma_load_3d(dst + kb * kBoxBytes, tk, full, 0, y, z);
-                            tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, tk, full, 64, y, z);
-                        }
+                    const int t = nk, nb = tl.boxes_in_tile(t);
+                    mbar_expect_tx(full, nb * 2u * kBoxBytes);
+                    for (int kb = 0; kb < nb; ++kb) {
+                        const int y = tl.box_start(tl.box_of(t, kb));
+                        tma_load_3d(dst + kb * kBoxBytes, tk, full, 0, y, z);
+                        tma_load_3d(dst + kHalfBytes + kb * kBoxBytes, tk, full, 64, y, z);
                     }
                     ++nk;
                     ++kq;
@@ -540,6 +548,7 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     }
     if (!ok) {
         // abort: let every copy already issued land before the CTA exits
+        if (qloads) wait_bar_quiet(sh.bar(B_QFULL), (qloads - 1) & 1);
         for (uint32_t s = 0; s < kKStages; ++s) {
             const uint32_t fills = kq / kKStages + (s < kq % kKStages ? 1u : 0u);
             if (fills) wait_bar_quiet(sh.bar(B_KFULL + s), (fills - 1) & 1);
@@ -557,25 +566,13 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
     const uint32_t idesc_pv = instr_desc(128, 128, true);
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t qp = 0, kq = 0, kv = 0, gt = 0;     // pieces, K-ring items, V tiles, tiles
+    uint32_t qp = 0, kq = 0, kv = 0, gt = 0;     // pieces, K tiles, V tiles, tiles
     bool ok = true;
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
-        {   // the piece's queries: K-ring item -> TMEM columns [kColQ, kColQ + 64)
-            const uint32_t st = kq % kKStages, n = kq / kKStages;
-            if (!wait_bar(sh.bar(B_KFULL + st), n & 1, sh.abort_flag, p.status) ||
-                (qp > 0 && !wait_bar(sh.bar(B_QEMPTY), (qp - 1) & 1, sh.abort_flag, p.status))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t qaddr = sh.base + kSmemK + st * kStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)      // 16 head dims per slice
-                tc_cp_128x256b(tmem + kColQ + 8 * kk,
-                               smem_desc(qaddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024));
-            tc_commit(sh.bar(B_KEMPTY + st));    // the slot is free once copied
-            ++kq;
+        if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) {
+            ok = false;
+            break;
         }
         // S(t) and PV(t) are issued as soon as their inputs are ready (S first
         // when both are: it feeds the softmax), so a late K tile does not hold
@@ -596,11 +593,13 @@ __device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, 
                     // one descriptor per tile; a step's is this one plus its byte
                     // offset / 16 (the 14-bit address field cannot carry out)
                     const uint64_t kd = smem_desc(sh.base + kSmemK + st * kStageBytes, 16, 1024);
+                    const uint64_t qd = smem_desc(sh.base + kSmemQ, 16, 1024);
                     const uint32_t dcol = tmem + buf * 128;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)     // 16 head dims per step; A = Q in TMEM
-                        tc_mma_ts(dcol, tmem + kColQ + 8 * kk, kd + (((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4),
-                                  idesc_s, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk) {   // 16 head dims per step
+                        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                        tc_mma_ss(dcol, qd + off, kd + off, idesc_s, kk > 0);
+                    }
                     tc_commit(sh.bar(B_SFULL + buf));
                     tc_commit(sh.bar(B_KEMPTY + st));
                     if (ns == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
@@ -1053,6 +1052,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- prologue: touches nothing an earlier kernel in the stream may write
     pdl_trigger();
     if (threadIdx.x == 0) {
+        mbar_init(sh.bar(B_QFULL), 1);
         mbar_init(sh.bar(B_QEMPTY), 1);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(sh.bar(B_KFULL + s), 1);
