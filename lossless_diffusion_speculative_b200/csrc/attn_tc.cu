@@ -49,8 +49,8 @@ namespace tc {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
+constexpr int kKStages = 2;
+constexpr int kVStages = 4;
 constexpr int kSBuf = 3;                    // S can run two tiles ahead of PV
 constexpr int kThreads = 192;
 constexpr int kBoxKeys = 64;
