@@ -28,10 +28,13 @@
 //                   a single bf16 P (2^-9) would break the 2e-3 * RMS tolerance
 //   O += P V        tcgen05.mma kind::f16 with A from TMEM, B = V tile (smem,
 //                   MN-major), N = 128 = head_dim, twice (hi, lo)
-// Roles: warps 0-3 softmax + output rows, warp 4 TMA producer, warp 5 MMA
-// issuer (+ TMEM allocation).  S is triple-buffered in TMEM (3 x 128 columns)
-// next to the O accumulator (128 columns); K and V have 3-stage smem rings;
-// after a piece the K ring stages the output rows for their bulk copies.
+// Roles: warps 0-3 softmax + output rows, warp 4 TMA producer, warp 5 S MMAs
+// (+ TMEM allocation), warp 6 PV MMAs (an MMA issue blocks its thread while
+// the tensor pipe is busy, so S and PV each get a thread of their own).
+// S is triple-buffered in TMEM (3 x 128 columns) next to the O accumulator
+// (128 columns); the query tile, two K stages and four V stages sit in shared
+// memory; after a piece the rings stage the output rows for their bulk
+// copies.
 // Launched with programmatic dependent launch: barrier setup, TMEM allocation
 // and descriptor prefetch overlap the previous kernel; nothing an earlier
 // kernel may write (ctx_lens, queries, cache, workspace) is read before
@@ -52,7 +55,7 @@ constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
 constexpr int kKStages = 2;
 constexpr int kVStages = 4;
 constexpr int kSBuf = 3;                    // S can run two tiles ahead of PV
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kBoxKeys = 64;
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B = 16 KiB
 constexpr uint32_t kQBytes = 2 * kHalfBytes;            // 128 query rows x 256 B
@@ -93,6 +96,7 @@ enum : int {
     B_MERGED,       // the piece's rows are out: the rings may be refilled
     B_GATHER,       // tx: the split partials of a segment have landed in smem
     B_DRAIN,
+    B_DRAIN2,
     B_COUNT
 };
 
@@ -560,110 +564,99 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
     }
 }
 
-__device__ __forceinline__ void mma_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                           int cid, uint32_t tmem)
+// Two MMA threads, each in its own warp, so that a batch of S MMAs and a
+// batch of PV MMAs are fed to the tensor pipe independently (an MMA issue
+// blocks its thread while the pipe is busy).
+//   S thread:  S(t) = Q K(t)^T once K(t) has landed and S buffer t % kSBuf is
+//              free again (PV(t - kSBuf) done)
+//   PV thread: O += P(t) V(t) once P(t) is written and V(t) has landed (the
+//              first PV of a piece also waits until the previous piece's O
+//              has been read out)
+__device__ __forceinline__ void s_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
+                                         int cid, uint32_t tmem)
 {
-    const uint32_t idesc_pv = instr_desc(128, 128, true);
     PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
     Piece pc;
-    uint32_t qp = 0, kq = 0, kv = 0, gt = 0;     // pieces, K tiles, V tiles, tiles
+    uint32_t qp = 0, kq = 0, gt = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
         const Tiling tl(pc.a, pc.e);
-        if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) {
-            ok = false;
-            break;
+        if (!wait_bar(sh.bar(B_QFULL), qp & 1, sh.abort_flag, p.status)) { ok = false; break; }
+        for (int t = 0; t < tl.ntile; ++t, ++kq, ++gt) {
+            const uint32_t st = kq % kKStages, n = kq / kKStages, buf = gt % kSBuf;
+            if (!wait_bar(sh.bar(B_KFULL + st), n & 1, sh.abort_flag, p.status) ||
+                (gt >= kSBuf && !wait_bar(sh.bar(B_PVDONE + buf), (gt / kSBuf - 1) & 1, sh.abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t idesc_s = instr_desc(128, 64 * tl.boxes_in_tile(t), false);
+            const uint64_t kd = smem_desc(sh.base + kSmemK + st * kStageBytes, 16, 1024);
+            const uint64_t qd = smem_desc(sh.base + kSmemQ, 16, 1024);
+            const uint32_t dcol = tmem + buf * 128;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {   // 16 head dims per step
+                const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                tc_mma_ss(dcol, qd + off, kd + off, idesc_s, kk > 0);
+            }
+            tc_commit(sh.bar(B_SFULL + buf));
+            tc_commit(sh.bar(B_KEMPTY + st));
+            if (t == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
         }
-        // S(t) and PV(t) are issued as soon as their inputs are ready (S first
-        // when both are: it feeds the softmax), so a late K tile does not hold
-        // back the PV of the tile before it
-        int ns = 0, npv = 0;
-        unsigned long long t0 = 0;
-        uint32_t idle = 0;
-        while (npv < tl.ntile) {
-            bool issued = false;
-            if (ns < tl.ntile) {       // S(ns) = Q K(ns)^T
-                const uint32_t st = (kq + ns) % kKStages, n = (kq + ns) / kKStages;
-                const uint32_t g = gt + ns, buf = g % kSBuf;
-                if (mbar_test(sh.bar(B_KFULL + st), n & 1) &&
-                    (g < kSBuf || mbar_test(sh.bar(B_PVDONE + buf), (g / kSBuf - 1) & 1))) {
-                    tc_fence_after();
-                    const int nb = tl.boxes_in_tile(ns);
-                    const uint32_t idesc_s = instr_desc(128, 64 * nb, false);
-                    // one descriptor per tile; a step's is this one plus its byte
-                    // offset / 16 (the 14-bit address field cannot carry out)
-                    const uint64_t kd = smem_desc(sh.base + kSmemK + st * kStageBytes, 16, 1024);
-                    const uint64_t qd = smem_desc(sh.base + kSmemQ, 16, 1024);
-                    const uint32_t dcol = tmem + buf * 128;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {   // 16 head dims per step
-                        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-                        tc_mma_ss(dcol, qd + off, kd + off, idesc_s, kk > 0);
-                    }
-                    tc_commit(sh.bar(B_SFULL + buf));
-                    tc_commit(sh.bar(B_KEMPTY + st));
-                    if (ns == tl.ntile - 1) tc_commit(sh.bar(B_QEMPTY));
-                    ++ns;
-                    issued = true;
-                }
-            }
-            if (!issued && npv < ns) {   // O += P(npv) V(npv)
-                const uint32_t st = (kv + npv) % kVStages, n = (kv + npv) / kVStages;
-                const uint32_t g = gt + npv, buf = g % kSBuf;
-                if (mbar_test(sh.bar(B_PFULL + buf), (g / kSBuf) & 1) && mbar_test(sh.bar(B_VFULL + st), n & 1) &&
-                    (npv > 0 || qp == 0 || mbar_test(sh.bar(B_OFREE), (qp - 1) & 1))) {
-                    tc_fence_after();
-                    // 16 keys per step (+2048 B of V, +8 columns of P); the issue
-                    // loops are unrolled with incremented descriptors so that the
-                    // single issuing thread keeps up with the tensor pipe
-                    const uint64_t vd = smem_desc(sh.base + kSmemV + st * kStageBytes, kHalfBytes, 1024);
-                    const uint32_t pcol = tmem + buf * 128, ocol = tmem + kColO;
-                    const uint32_t acc0 = npv == 0 ? 0u : 1u;
-                    if (tl.boxes_in_tile(npv) == 2) {
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
-                    }
-                    tc_commit(sh.bar(B_VEMPTY + st));
-                    tc_commit(sh.bar(B_PVDONE + buf));
-                    ++npv;
-                    issued = true;
-                }
-            }
-            if (issued) {
-                idle = 0;
-            } else {                    // bounded: the same limit as wait_bar
-                if (idle == 0) t0 = global_ns();
-                if ((++idle & 63u) == 0) {
-                    if (*sh.abort_flag) { ok = false; break; }
-                    if (global_ns() - t0 > kTimeoutNs) {
-                        *sh.abort_flag = 1;
-                        raise_status(p.status, ORTHRUS_STATUS_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                }
-                __nanosleep(20);
-            }
-        }
-        kq += tl.ntile;
-        kv += tl.ntile;
-        gt += tl.ntile;
         ++qp;
     }
     if (!ok) {                          // abort: wait for every MMA issued so far
         tc_commit(sh.bar(B_DRAIN));
         wait_bar_quiet(sh.bar(B_DRAIN), 0);
+    }
+}
+
+__device__ __forceinline__ void pv_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
+                                          int cid, uint32_t tmem)
+{
+    const uint32_t idesc_pv = instr_desc(128, 128, true);
+    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
+    Piece pc;
+    uint32_t qp = 0, kv = 0, gt = 0;
+    bool ok = true;
+    while (ok && it.next(pc)) {
+        const Tiling tl(pc.a, pc.e);
+        for (int t = 0; t < tl.ntile; ++t, ++kv, ++gt) {
+            const uint32_t st = kv % kVStages, n = kv / kVStages, buf = gt % kSBuf;
+            if (!wait_bar(sh.bar(B_PFULL + buf), (gt / kSBuf) & 1, sh.abort_flag, p.status) ||
+                !wait_bar(sh.bar(B_VFULL + st), n & 1, sh.abort_flag, p.status) ||
+                (t == 0 && qp > 0 && !wait_bar(sh.bar(B_OFREE), (qp - 1) & 1, sh.abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // 16 keys per step (+2048 B of V, +8 columns of P)
+            const uint64_t vd = smem_desc(sh.base + kSmemV + st * kStageBytes, kHalfBytes, 1024);
+            const uint32_t pcol = tmem + buf * 128, ocol = tmem + kColO;
+            const uint32_t acc0 = t == 0 ? 0u : 1u;
+            if (tl.boxes_in_tile(t) == 2) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_ts(ocol, pcol + 8 * kk, vd + kk * 128, idesc_pv, kk == 0 ? acc0 : 1u);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_ts(ocol, pcol + 64 + 8 * kk, vd + kk * 128, idesc_pv, 1u);
+            }
+            tc_commit(sh.bar(B_VEMPTY + st));
+            tc_commit(sh.bar(B_PVDONE + buf));
+        }
+        ++qp;
+    }
+    if (!ok) {
+        tc_commit(sh.bar(B_DRAIN2));
+        wait_bar_quiet(sh.bar(B_DRAIN2), 0);
     }
 }
 
@@ -1072,6 +1065,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(sh.bar(B_MERGED), 1);
         mbar_init(sh.bar(B_GATHER), 1);
         mbar_init(sh.bar(B_DRAIN), 1);
+        mbar_init(sh.bar(B_DRAIN2), 1);
         *sh.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1106,8 +1100,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == 4) {
             if (lane == 0) producer(sh, p, d, cid, &tm_q, &tm_k, &tm_v);
             __syncwarp();
+        } else if (warp == 5) {
+            if (lane == 0) s_issuer(sh, p, d, cid, tmem);
+            __syncwarp();
         } else {
-            if (lane == 0) mma_issuer(sh, p, d, cid, tmem);
+            if (lane == 0) pv_issuer(sh, p, d, cid, tmem);
             __syncwarp();
         }
     }
