@@ -316,13 +316,52 @@ def main():
             d2h = 2 * w.B * 4
             e_steps = max(1, min(args.steps, 500))
 
+            # The copies of a step go out on their own stream in the order the
+            # step consumes them (per group of layers: block K/V and queries of
+            # the DIFF view, then the same of the AR view, then logits and
+            # proposals); the step runs as graphs of those layer groups and each
+            # waits only for what it reads.  A step's copies start once the
+            # previous step is done with the buffers.
+            cs = torch.cuda.Stream(device=dev)
+            chunk = 9
+            egraphs = None if graphs is None else st.capture(stream, chunk=chunk)
+            chunks, needs = [], {}
+            if args.order == "cold":
+                for view, vn in ((0, "diff"), (1, "ar")):
+                    for c in range(0, st.L, chunk):
+                        sl = (view, slice(c, min(c + chunk, st.L)))
+                        needs[f"write_block_{vn}_{c}"] = needs[f"attn_{vn}_{c}"] = len(chunks)
+                        chunks.append([("kb", sl), ("vb", sl), ("q", sl)])
+            else:
+                needs["attn_interleaved"] = len(chunks)
+                chunks.append([("kb", None), ("vb", None), ("q", None)])
+            needs["consensus_commit"] = len(chunks)
+            chunks.append([("logits", None), ("proposed", None)])
+            ready = [torch.cuda.Event() for _ in chunks]
+            done = torch.cuda.Event()
+
             def e2e_step():
-                for n in host:
-                    dst[n].copy_(host[n], non_blocking=True)
-                one_step()
+                if graphs is None:
+                    for n in host:
+                        dst[n].copy_(host[n], non_blocking=True)
+                    one_step()
+                else:
+                    cs.wait_event(done)
+                    with torch.cuda.stream(cs):
+                        for ev_i, ch in zip(ready, chunks):
+                            for n, v in ch:
+                                d_t, h_t = (dst[n], host[n]) if v is None else (dst[n][v], host[n][v])
+                                d_t.copy_(h_t, non_blocking=True)
+                            ev_i.record(cs)
+                    egraphs[0][1].replay()
+                    for name, g in egraphs[1:]:
+                        stream.wait_event(ready[needs[name]])
+                        g.replay()
                 out_acc.copy_(st.accepted, non_blocking=True)
                 out_nxt.copy_(st.next_token, non_blocking=True)
+                done.record(stream)
 
+            done.record(stream)
             for _ in range(3):
                 e2e_step()
             torch.cuda.synchronize()
@@ -330,6 +369,7 @@ def main():
             a0 = torch.cuda.Event(enable_timing=True)
             a1 = torch.cuda.Event(enable_timing=True)
             a0.record()
+            done.record(stream)
             for _ in range(e_steps):
                 e2e_step()
             a1.record()

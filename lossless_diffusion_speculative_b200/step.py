@@ -84,10 +84,11 @@ class DecodeStep:
         self.tc_path = ob.orthrus_attn_path(B, Hq, Hkv, D, K, dt) == 1
 
     # -- the hot path, as launch sequences ---------------------------------
-    def _write_block(self, view):
-        ob.orthrus_write_block(self.ctx, self.k_cache, self.v_cache,
-                               [self.kb_all[view, l] for l in range(self.L)],
-                               [self.vb_all[view, l] for l in range(self.L)], status=self.status)
+    def _write_block(self, view, layers=None):
+        layers = range(self.L) if layers is None else layers
+        ob.orthrus_write_block(self.ctx, [self.k_cache[l] for l in layers], [self.v_cache[l] for l in layers],
+                               [self.kb_all[view, l] for l in layers],
+                               [self.vb_all[view, l] for l in layers], status=self.status)
 
     def _attn(self, view, layer):
         ob.orthrus_attn(view, self.q_all[view, layer], self.k_cache[layer], self.v_cache[layer],
@@ -104,8 +105,23 @@ class DecodeStep:
         ob.orthrus_kv_commit(self.ctx, self.accepted, K=w.K, Hkv=w.Hkv, D=w.D, S_max=w.S_max,
                              dtype=self.dtype, num_layers=self.L, status=self.status)
 
-    def segments(self):
-        """The step as ordered launch segments (timed separately by the bench)."""
+    def segments(self, chunk: int = 0):
+        """The step as ordered launch segments (timed separately by the bench).
+
+        With ``chunk`` > 0 (cold order) each view runs as layer groups of that
+        size, block install then attention per group: the same launches' work in
+        smaller segments, so that a caller feeding the step from the host can
+        start each group once its inputs have arrived.
+        """
+        if self.order == "cold" and chunk > 0:
+            segs = []
+            for view, vn in ((ob.DIFF, "diff"), (ob.AR, "ar")):
+                for c in range(0, self.L, chunk):
+                    layers = range(c, min(c + chunk, self.L))
+                    segs.append((f"write_block_{vn}_{c}", lambda v=view, ls=layers: self._write_block(v, ls)))
+                    segs.append((f"attn_{vn}_{c}", lambda v=view, ls=layers: [self._attn(v, l) for l in ls]))
+            segs.append(("consensus_commit", self._tail))
+            return segs
         if self.order == "cold":
             return [("write_block_diff", lambda: self._write_block(ob.DIFF)),
                     ("attn_diff", lambda: self._attn_view(ob.DIFF)),
@@ -130,7 +146,7 @@ class DecodeStep:
         for _, fn in self.segments():
             fn()
 
-    def capture(self, stream: torch.cuda.Stream):
+    def capture(self, stream: torch.cuda.Stream, chunk: int = 0):
         """CUDA graphs of the reset and of every segment (captured on ``stream``)."""
         self.run_eager()                    # warm: attributes set, plans cached
         torch.cuda.synchronize()
@@ -140,7 +156,7 @@ class DecodeStep:
             with torch.cuda.graph(g, stream=stream):
                 self.reset()
             graphs.append(("reset", g))
-            for name, fn in self.segments():
+            for name, fn in self.segments(chunk):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
                     fn()
