@@ -141,14 +141,14 @@ class DecodeStep:
     def reset(self):
         self.ctx.copy_(self.ctx0, non_blocking=True)
 
-    def run_eager(self):
+    def run_eager(self, chunk: int = 0):
         self.reset()
-        for _, fn in self.segments():
+        for _, fn in self.segments(chunk):
             fn()
 
     def capture(self, stream: torch.cuda.Stream, chunk: int = 0):
         """CUDA graphs of the reset and of every segment (captured on ``stream``)."""
-        self.run_eager()                    # warm: attributes set, plans cached
+        self.run_eager(chunk)               # warm: attributes set, plans cached
         torch.cuda.synchronize()
         graphs = []
         with torch.cuda.stream(stream):

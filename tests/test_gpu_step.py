@@ -14,20 +14,22 @@ from gpu_util import assert_attn_close
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("order", ["cold", "interleaved"])
+@pytest.mark.parametrize("order,chunk", [("cold", 0), ("interleaved", 0), ("cold", 2)])
 @pytest.mark.parametrize("graph", [False, True])
-def test_step_matches_oracle(order, graph):
+def test_step_matches_oracle(order, chunk, graph):
+    # chunk > 0: each view as layer groups (install, then attention, per group),
+    # the segmentation the end-to-end benchmark feeds from the host
     w = wl.WORKLOADS["qwen3_8b_step"].with_(ctx_lo=1500, ctx_hi=1500, layers=3,
                                             plant="fixed:9")
     st = DecodeStep(w, order=order)
     if graph:
         s = torch.cuda.Stream()
-        graphs = st.capture(s)
+        graphs = st.capture(s, chunk=chunk)
         with torch.cuda.stream(s):
             for _, g in graphs:
                 g.replay()
     else:
-        st.run_eager()
+        st.run_eager(chunk)
     res = st.result()
     assert int(st.status.item()) == 0
     ci = st.consensus_in
