@@ -60,9 +60,12 @@ AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int K, orthrus_dtype dt, int s
     }
     pl.slots = pl.grid + B * Hkv;
     // equal-length segments split evenly when the unit count is a multiple of
-    // the segment count (no unit straddles a segment boundary)
+    // the segment count (no unit straddles a segment boundary): rounded down
+    // to one when that idles at most 1/16 of the units; otherwise every unit
+    // works and some straddle two segments (ragged lengths gain nothing from
+    // the rounding either)
     const int segs = B * Hkv;
-    if (pl.grid >= segs) pl.grid -= pl.grid % segs;
+    if (pl.grid >= segs && pl.grid % segs <= pl.grid / 16) pl.grid -= pl.grid % segs;
     return pl;
 }
 
