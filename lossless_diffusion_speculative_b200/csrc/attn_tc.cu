@@ -77,7 +77,8 @@ static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemBar, "staging rows fi
 // kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
 // two weight rows per warp (8 x n floats)
 constexpr uint32_t kSmemGather = kSmemQ;
-static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
+constexpr int kLseOneCopy = 16384;                      // bytes: the lse rows of all partials in one copy
+static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + kLseOneCopy + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
                       8 * kMaxSyncUnits * 4 <= kSmemBar,
               "split merge fits in the rings");
 
@@ -674,17 +675,27 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
     for (int ch = 0; ch < 4; ++ch) {
         if (ch < 2 * nb) {
             uint32_t hi[16], lo[16];
+            float2 pe[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                pe[j] = ffma2(make_float2(__uint_as_float(s[32 * ch + 2 * j]),
+                                          __uint_as_float(s[32 * ch + 2 * j + 1])),
+                              sc, nm);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pe[j] = make_float2(fast_exp2(pe[j].x), fast_exp2(pe[j].y));
+            float2 l2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                lsum = fadd2(lsum, pe[j]);
+                l2 = fadd2(l2, pe[j + 1]);
+            }
+            lsum = fadd2(lsum, l2);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float2 x = ffma2(make_float2(__uint_as_float(s[32 * ch + 2 * j]),
-                                                   __uint_as_float(s[32 * ch + 2 * j + 1])),
-                                       sc, nm);
-                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-                lsum = fadd2(lsum, pe);
-                const uint32_t u0 = __float_as_uint(pe.x), u1 = __float_as_uint(pe.y);
+                const uint32_t u0 = __float_as_uint(pe[j].x), u1 = __float_as_uint(pe[j].y);
                 hi[j] = __byte_perm(u0, u1, 0x7632);
-                const float2 r = fsub2(pe, make_float2(__uint_as_float(u0 & 0xFFFF0000u),
-                                                       __uint_as_float(u1 & 0xFFFF0000u)));
+                const float2 r = fsub2(pe[j], make_float2(__uint_as_float(u0 & 0xFFFF0000u),
+                                                          __uint_as_float(u1 & 0xFFFF0000u)));
                 lo[j] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
             }
             tmem_st16(p_addr + 16 * ch, hi);
@@ -713,7 +724,12 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
     const int lp = lse_pitch(rows);
     const int j = cid - sp.c_lo;
     const int r_lo = j * rows / sp.n, nr = (j + 1) * rows / sp.n - r_lo;
-    const int l_lo = r_lo & ~3, nl = ((r_lo + nr + 3) & ~3) - l_lo;   // 16-byte lse rows
+    // log2-sum-exp values: when the n partials' whole lse rows are small
+    // (n * lp floats, contiguous in the workspace) one bulk copy brings them
+    // all, else each partial's 16-byte-aligned run covering this CTA's rows
+    const bool one_lse = sp.n * lp * 4 <= kLseOneCopy;
+    const int l_lo = one_lse ? 0 : r_lo & ~3;
+    const int nl = one_lse ? lp : ((r_lo + nr + 3) & ~3) - l_lo;     // lse floats per partial
     const uint32_t o_bytes = (uint32_t)nr * kD * 4, l_bytes = (uint32_t)nl * 4;
     const uint32_t s_lse = kSmemGather + (uint32_t)sp.n * o_bytes;     // after the O rows
     const uint32_t s_w = s_lse + (((uint32_t)sp.n * l_bytes + 15u) & ~15u);   // [4 warps][2][n] weights
@@ -737,12 +753,15 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
         // it, and the proxy fence orders the bulk reads after both)
         __syncwarp();
         fence_proxy_async_global();
-        if (nr > 0)
+        if (nr > 0) {
             for (int q = lane; q < sp.n; q += 32) {
                 const size_t slot = (size_t)sp.c_lo + q + sp.s;
                 bulk_load(base + kSmemGather + q * o_bytes, ws_o + (slot * rows + r_lo) * kD, o_bytes, bar);
-                bulk_load(base + s_lse + q * l_bytes, ws_lse + slot * lp + l_lo, l_bytes, bar);
+                if (!one_lse) bulk_load(base + s_lse + q * l_bytes, ws_lse + slot * lp + l_lo, l_bytes, bar);
             }
+            if (one_lse && lane == 0)
+                bulk_load(base + s_lse, ws_lse + ((size_t)sp.c_lo + sp.s) * lp, (uint32_t)sp.n * l_bytes, bar);
+        }
         if (lane == 0 && counter_fetch_add_acq_rel(ws_sync + kMaxSyncUnits + sp.c_lo, 1) == sp.n - 1) {
             arrive[0] = 0;                                    // everyone has passed the wait
             ws_sync[kMaxSyncUnits + sp.c_lo] = 0;
