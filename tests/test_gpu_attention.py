@@ -186,3 +186,28 @@ def test_workspace_reused_across_calls_and_shapes():
             assert int(ws[:1280].count_nonzero().item()) == 0, "split-merge counters left set"
             assert_attn_close(out.cpu().numpy(), oracle.attention(view, q, kc, vc, ctx),
                               f"reuse B={B} view={view}")
+
+
+def test_merge_wait_gives_up_on_counters_that_never_complete():
+    """A workspace whose split-merge counters were not zeroed (documented
+    misuse): every split segment's merge waits for a count that can never
+    arrive, gives up after its bound, and the call sets ORTHRUS_STATUS_TIMEOUT
+    instead of hanging or faulting; the context stays usable and the next call
+    on a zeroed workspace is exact."""
+    q, kc, vc, ctx = _custom(15, 1, 32, 8, 128, 32, [5000])     # every segment split
+    args = [to_dev(x, torch.bfloat16) for x in (q, kc, vc)]
+    c = torch.from_numpy(ctx).cuda()
+    need = ob.orthrus_attn_workspace_size(1, 32, 8, 128, 32, torch.bfloat16)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws[:640].view(torch.int32).fill_(-1_000_000)                # arrive counters
+    out = torch.empty((1, 32, 32, 128), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ob.orthrus_attn(ob.DIFF, *args, c, out, ws, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & ob.STATUS_TIMEOUT
+    ws.zero_()
+    status.zero_()
+    ob.orthrus_attn(ob.DIFF, *args, c, out, ws, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_attn_close(out.cpu().numpy(), oracle.attention(ob.DIFF, q, kc, vc, ctx), "after timeout")
