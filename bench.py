@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qwen3_8b_step] [--order cold|interleaved] [--no-graph]
+                    [--no-e2e] [--no-cpu-baseline] [--no-configs]
 
 One step = block install + attention of the diffusion view over every layer,
 block install + attention of the AR verification view over every layer, the
@@ -16,10 +17,15 @@ other layer has streamed through.
 Prints ONE JSON line (rank 0).  ``value`` is verified tokens/s over all ranks:
 sum over ranks of (tokens committed per step x steps) / max-over-ranks time.
 Multi-GPU runs are independent replicas (data parallel, no collective on the
-data path; "scaling": "weak").
+data path; "scaling": "weak").  The line also carries a ``configs`` block: the
+attention of both views, KV-read bandwidth and its fraction of the measured HBM
+bandwidth, and verified tokens/s for every workload of the decode step (medians
+of at least 50 L2-cold iterations each).
 
-``--impl reference`` times the fp64 CPU oracle on the host cores instead, each
-step a bounded sample of the same workload extrapolated to a full step.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead: each
+step runs whole layer-view attentions (every output row) of the same workload,
+as many as keep the whole run within a few minutes (all 72 of a step at the
+default driver settings), plus the consensus when the step is complete.
 """
 from __future__ import annotations
 
@@ -41,11 +47,24 @@ sys.path.insert(0, ROOT)
 METRIC = ("dual-view decode-step attn µs & KV-read GB/s vs 8 TB/s; verified tokens/s")
 UNIT = "verified tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
+CONFIG_ITERS = 60                   # per configuration of the configs block
+REF_BUDGET_S = 150.0                # reference arm: timed CPU seconds per run
 
 # DRAM traffic of one attn_tc_kernel launch on the headline workload, from the
 # ncu capture summarised in profiles/ (bytes read + written), keyed by the hash
 # of the kernel source it was taken on; reported as null once the source changes.
 NCU_TRAFFIC = {("qwen3_8b_step", "3a5dfd49b7df8d12"): 34.05e6}
+
+# The workloads of the configs block: (label, workload, order).  The 36-layer
+# step in its specified per-layer order (DIFF then AR per layer) is timed in
+# full; the others are single attention layers.
+CONFIG_SET = (("qwen3_1p7b_layer", "qwen3_1p7b_layer", "cold"),
+              ("qwen3_8b_step_interleaved", "qwen3_8b_step", "interleaved"),
+              ("qwen3_4b_ragged", "qwen3_4b_ragged", "cold"),
+              ("qwen3_8b_long_k8", "qwen3_8b_long_k8", "cold"),
+              ("qwen3_8b_long_k16", "qwen3_8b_long_k16", "cold"),
+              ("qwen3_8b_long_k32", "qwen3_8b_long_k32", "cold"))
 
 
 def parse():
@@ -59,6 +78,7 @@ def parse():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     return ap.parse_args()
 
 
@@ -80,7 +100,9 @@ def kernel_hash():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons."""
+    """nvidia-smi samples (100 ms) of SM clock, power and throttle reasons,
+    from the first warm-up step to the end of the last GPU leg.  Samples whose
+    power draw shows the GPU busy count as "under load"."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -94,7 +116,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -107,57 +129,68 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons = [], None, set()
+        rows = []
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax = float(parts[1])
+                sm, smax, pw = float(parts[0]), float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            active = {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}
+            rows.append((sm, smax, pw, active))
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        idle = min(r[2] for r in rows)
+        load = [r for r in rows if r[2] >= idle + 100.0] or rows
+        reasons = sorted(set().union(*[r[3] for r in load]))
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": rows[-1][1],
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r[2] for r in rows),
+                "window": "first warm-up step to the end of the last GPU leg"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_step_estimate(w, budget_s: float, n_threads: int = 0):
-    """Time the fp64 oracle on a bounded sample of one decode step and scale it
-    to a full step.  Returns (seconds per full step, sample description, threads)."""
-    import oracle
-    from lossless_diffusion_speculative_b200 import workloads as wl
-    n_views = 2 * w.layers
-    t_attn, done = 0.0, 0
-    for layer in range(w.layers):
-        for view in (0, 1):
-            li = wl.layer_inputs(w, layer, view, poison=False)
-            t0 = time.perf_counter()
-            oracle.attention(view, li.q, li.k_cache, li.v_cache, li.ctx_lens, n_threads=n_threads)
-            t_attn += time.perf_counter() - t0
-            done += 1
-            if t_attn >= budget_s:
-                break
-        if t_attn >= budget_s:
-            break
-    ci = wl.consensus_inputs(w)
-    t0 = time.perf_counter()
-    oracle.consensus(ci.logits, ci.proposed)
-    t_cons = time.perf_counter() - t0
-    step_s = t_attn / done * n_views + t_cons
-    desc = (f"{done} of {n_views} layer-view attentions (all rows) + full consensus, "
-            f"scaled to {n_views} layer-views")
-    return step_s, desc, oracle.num_threads() if n_threads <= 0 else n_threads
+class OracleStep:
+    """One decode step of the fp64 oracle: 2 x layers whole layer-view
+    attentions (every output row, all host threads) and the consensus.
+
+    The attention inputs of layer 0 (both views) stand in for every layer: the
+    oracle's cost depends on the shapes only (its loops have no data-dependent
+    trip counts), and regenerating 36 seeded caches per step would dominate the
+    run with untimed input generation."""
+
+    def __init__(self, w):
+        from lossless_diffusion_speculative_b200 import workloads as wl
+        self.w = w
+        self.li = [wl.layer_inputs(w, 0, v, poison=False) for v in (0, 1)]
+        self.ci = wl.consensus_inputs(w)
+        self.n_views = 2 * w.layers
+
+    def layer_view(self, j: int) -> None:
+        import oracle
+        li = self.li[j % 2]
+        oracle.attention(j % 2, li.q, li.k_cache, li.v_cache, li.ctx_lens)
+
+    def consensus(self) -> None:
+        import oracle
+        oracle.consensus(self.ci.logits, self.ci.proposed)
+
+    def full_step(self) -> float:
+        t0 = time.perf_counter()
+        for j in range(self.n_views):
+            self.layer_view(j)
+        self.consensus()
+        return time.perf_counter() - t0
 
 
 def run_reference(args, w, rank, world):
@@ -166,38 +199,48 @@ def run_reference(args, w, rank, world):
         return
     import oracle
     from lossless_diffusion_speculative_b200 import workloads as wl
-    li = [wl.layer_inputs(w, 0, v, poison=False) for v in (0, 1)]
-    ci = wl.consensus_inputs(w)
+    os_ = OracleStep(w)
     t0 = time.perf_counter()
-    oracle.consensus(ci.logits, ci.proposed)
-    t_cons = time.perf_counter() - t0
-    rows_total = w.B * w.K * w.Hq
-    # each step: R rows of one view's attention; sized so K steps take ~minutes
-    R = 32
-    rng = np.random.default_rng(0)
-    times = []
-    for s in range(args.warmup + args.steps):
-        view = s % 2
-        rows = np.stack([rng.integers(0, w.B, R), rng.integers(0, w.K, R),
-                         rng.integers(0, w.Hq, R)], axis=1).astype(np.int32)
+    os_.layer_view(0)                                   # first call: sizes the sample
+    t_lv = time.perf_counter() - t0
+    per_step = int(min(os_.n_views, max(1, REF_BUDGET_S / max(1, args.steps) / t_lv)))
+    full = per_step == os_.n_views
+    for s in range(args.warmup):                        # untimed, one layer-view each
+        os_.layer_view(s)
+    times, lv_times = [], []
+    for s in range(args.steps):
         t0 = time.perf_counter()
-        oracle.attention(view, li[view].q, li[view].k_cache, li[view].v_cache,
-                         li[view].ctx_lens, rows=rows)
-        dt = time.perf_counter() - t0
-        if s >= args.warmup:
-            times.append(dt)
-    t_rows = float(np.mean(times))
-    step_s = t_rows * (rows_total / R) * 2 * w.layers + t_cons
-    tokens = int(np.minimum(ci.planted_accept + 1, w.K).sum())
+        for j in range(per_step):
+            os_.layer_view(s * per_step + j)
+        t1 = time.perf_counter()
+        if full:
+            os_.consensus()
+        t2 = time.perf_counter()
+        times.append(t2 - t0)
+        lv_times.append((t1 - t0) / per_step)
+    tokens = int(np.minimum(os_.ci.planted_accept + 1, w.K).sum())
+    tokens_exp = wl.expected_tokens_per_step(w)
+    if full:
+        step_s = float(np.median(times))
+        sample = (f"every step: all {os_.n_views} layer-view attentions (all rows) + the "
+                  "consensus over the full vocabulary; median step time")
+    else:
+        t0 = time.perf_counter()
+        os_.consensus()
+        t_cons = time.perf_counter() - t0
+        step_s = float(np.median(lv_times)) * os_.n_views + t_cons
+        sample = (f"every step: {per_step} of {os_.n_views} layer-view attentions (all rows); "
+                  "a full step = median layer-view time x "
+                  f"{os_.n_views} + one consensus ({t_cons * 1e3:.0f} ms)")
     value = tokens / step_s
-    sample = (f"per step {R} random attention rows of layer 0 (alternating views) of "
-              f"{rows_total} rows x {2 * w.layers} layer-views, + one full consensus; "
-              "scaled to a full step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": float(np.mean(times)) * 1e3,
+            "ms_per_full_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": config_of(w, args),
+            "tokens_per_step": tokens, "tokens_per_step_expected": tokens_exp,
+            "value_at_expected_tokens": tokens_exp / step_s,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -211,9 +254,61 @@ def config_of(w, args):
             "layers": w.layers, "ctx": int(ctx[0]) if w.ctx_lo == w.ctx_hi else
             [int(ctx.min()), int(ctx.max())], "K": w.K, "vocab": w.vocab,
             "order": args.order, "graphs": not args.no_graph,
-            "l2": "inputs larger than L2: each step streams every layer's KV cache "
-                  f"({w.kv_bytes_per_view_layer() * 2 * w.layers / 1e9:.2f} GB) through the "
-                  "126 MB L2"}
+            "l2": ("inputs larger than L2: each step streams every layer's KV cache "
+                   f"({w.kv_bytes_per_view_layer() * 2 * w.layers / 1e9:.2f} GB) through the "
+                   "126 MB L2") if w.kv_bytes_per_view_layer() * w.layers > L2_FLUSH_BYTES // 2
+            else "KV cache fits in L2: the configs block flushes L2 before every attention"}
+
+
+# ----------------------------------------------------------------------------- configs block
+def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
+    """Median µs of each launch segment of one workload's step over `iters`
+    replays, L2 flushed before every attention segment (outside the events).
+    `st` reuses an existing DecodeStep of the same workload."""
+    import torch
+    from lossless_diffusion_speculative_b200.step import DecodeStep
+
+    if st is None:
+        st = DecodeStep(w, order=order, device=dev)
+    graphs = st.capture(stream, order=order)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    names = [n for n, _ in graphs[1:]]
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in names] for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for it in range(3 + iters):
+            graphs[0][1].replay()
+            for k, (name, g) in enumerate(graphs[1:]):
+                if name.startswith("attn"):
+                    flush.zero_()
+                if it >= 3:
+                    ev[it - 3][k][0].record()
+                g.replay()
+                if it >= 3:
+                    ev[it - 3][k][1].record()
+        torch.cuda.synchronize()
+    if int(st.status.item()) != 0:
+        raise RuntimeError(f"{label}: device status {int(st.status.item()):#x}")
+    med = {n: float(np.median([ev[i][k][0].elapsed_time(ev[i][k][1]) for i in range(iters)]))
+           * 1e3 for k, n in enumerate(names)}
+    attn_us = sum(v for n, v in med.items() if n.startswith("attn"))
+    step_us = sum(med.values())
+    kv = st.kv_bytes_per_attn_call() * 2 * st.L
+    gbs = kv / (attn_us * 1e-6) / 1e9
+    tok, tok_e = st.tokens_per_step(), st.tokens_per_step_expected()
+    calls = 2 * st.L
+    out = {"workload": w.name, "order": order, "B": w.B, "K": w.K, "layers": st.L,
+           "ctx": [int(w.ctx_lens().min()), int(w.ctx_lens().max())],
+           "attn_us": attn_us, "attn_us_per_call": attn_us / calls,
+           "kv_bytes_per_step": kv, "kv_read_gbs": gbs, "kv_read_frac_of_hbm": gbs / hbm,
+           "kv_read_frac_of_8tbs": gbs / 8000.0, "step_us": step_us,
+           "tokens_per_step": tok, "tokens_per_step_expected": tok_e,
+           "verified_tokens_per_s": tok / (step_us * 1e-6),
+           "verified_tokens_per_s_at_expected": tok_e / (step_us * 1e-6),
+           "segments_us": med, "iters": iters,
+           "timing": "median of per-segment CUDA events; L2 flushed before each attention segment"}
+    del graphs, st
+    return out
 
 
 # ----------------------------------------------------------------------------- main
@@ -241,10 +336,13 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
+    hbm, hbm_src = peaks()
     st = DecodeStep(w, order=args.order, device=dev)
     stream = torch.cuda.Stream(device=dev)
     graphs = None if args.no_graph else st.capture(stream)
     segs = [n for n, _ in st.segments()]
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
 
     def one_step(evs=None):
         if graphs is None:
@@ -269,6 +367,7 @@ def main():
             dist.barrier()
 
     with torch.cuda.stream(stream):
+        sampler.start()
         for _ in range(args.warmup):
             one_step()
         torch.cuda.synchronize()
@@ -278,11 +377,8 @@ def main():
         nseg = len(segs)
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nseg + 1)]
               for _ in range(args.steps)]
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
         barrier()
         torch.cuda.synchronize()
-        sampler.start()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record()
@@ -290,14 +386,12 @@ def main():
             one_step(ev[s])
         t_end.record()
         torch.cuda.synchronize()
-        clocks = sampler.stop()
         barrier()
         elapsed_ms = t_start.elapsed_time(t_end)
-        seg_ms = np.zeros(nseg)
+        seg_ms = np.zeros((args.steps, nseg))
         for s in range(args.steps):
             for i in range(nseg):
-                seg_ms[i] += ev[s][i].elapsed_time(ev[s][i + 1])
-        seg_ms /= args.steps
+                seg_ms[s, i] = ev[s][i].elapsed_time(ev[s][i + 1])
 
         # ---- end to end: host inputs in (pinned), result out, every step
         e2e = None
@@ -378,19 +472,34 @@ def main():
             e2e_ms = a0.elapsed_time(a1)
             assert int(out_acc[0]) == int(res.accepted[0])
             e2e = (e2e_ms, e_steps, h2d, d2h)
+            egraphs = None
+
+        # ---- every workload of the decode step, one at a time (rank 0 only)
+        configs = None
+        if rank == 0 and world == 1 and not args.no_configs:
+            configs = {}
+            for label, name, order in CONFIG_SET:
+                configs[label] = measure_config(label, wl.WORKLOADS[name], order, dev, stream,
+                                                hbm, CONFIG_ITERS,
+                                                st=st if name == w.name else None)
+                torch.cuda.empty_cache()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
 
     # ---- max over ranks (independent replicas: no data-path collective)
     elapsed_ms, e2e_ms_max = max_over_ranks([elapsed_ms, e2e[0] if e2e else 0.0], device=dev)
 
     tokens = st.tokens_per_step()
+    tokens_exp = st.tokens_per_step_expected()
     ms_per_step = elapsed_ms / args.steps
     value = replica_throughput(tokens, args.steps, world, elapsed_ms)
     kv_step = st.kv_bytes_per_attn_call() * 2 * st.L
-    hbm, hbm_src = peaks()
     if args.order == "cold":
-        attn_ms = seg_ms[segs.index("attn_diff")] + seg_ms[segs.index("attn_ar")]
+        attn_ms_steps = seg_ms[:, segs.index("attn_diff")] + seg_ms[:, segs.index("attn_ar")]
     else:
-        attn_ms = seg_ms[segs.index("attn_interleaved")]
+        attn_ms_steps = seg_ms[:, segs.index("attn_interleaved")]
+    attn_ms = float(np.mean(attn_ms_steps))
+    attn_ms_med = float(np.median(attn_ms_steps))
     per_call_s = attn_ms / 1e3 / (2 * st.L)
     achieved = st.kv_bytes_per_attn_call() / per_call_s / 1e9
     traffic = NCU_TRAFFIC.get((w.name, kernel_hash()))
@@ -402,15 +511,20 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "ms_per_step_median": float(np.median(seg_ms.sum(axis=1))),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded Qwen3-shaped tensors; planted acceptance)",
             "config": config_of(w, args),
             "tokens_per_step": tokens,
+            "tokens_per_step_expected": tokens_exp,
+            "value_at_expected_tokens": replica_throughput(tokens_exp, args.steps, world,
+                                                           elapsed_ms),
             "attn_us_per_step": attn_ms * 1e3,
+            "attn_us_per_step_median": attn_ms_med * 1e3,
             "kv_read_gbs": kv_step / (attn_ms / 1e3) / 1e9,
             "kv_read_frac_of_hbm": kv_step / (attn_ms / 1e3) / 1e9 / hbm,
             "kv_read_frac_of_8tbs": kv_step / (attn_ms / 1e3) / 1e9 / 8000.0,
-            "segments_us": {n: float(v * 1e3) for n, v in zip(segs, seg_ms)},
+            "segments_us": {n: float(v * 1e3) for n, v in zip(segs, seg_ms.mean(axis=0))},
             "attn_path": "tcgen05" if st.tc_path else "cuda-core",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
@@ -425,10 +539,16 @@ def main():
             line["e2e"] = {"value": replica_throughput(tokens, e2e[1], world, e2e_ms_max), "unit": UNIT,
                            "h2d_bytes_per_step": e2e[2], "d2h_bytes_per_step": e2e[3],
                            "steps": e2e[1]}
+        if configs:
+            line["configs"] = configs
         if world == 1 and not args.no_cpu_baseline:
-            step_s, desc, cores = oracle_step_estimate(w, budget_s=10.0)
-            line["cpu_baseline"] = {"value": tokens / step_s, "unit": UNIT, "cores": cores,
-                                    "kind": "oracle", "sample": desc,
+            os_ = OracleStep(w)
+            step_s = os_.full_step()
+            import oracle
+            line["cpu_baseline"] = {"value": tokens / step_s, "unit": UNIT,
+                                    "cores": oracle.num_threads(), "kind": "oracle",
+                                    "sample": f"one full decode step: all {os_.n_views} "
+                                              "layer-view attentions (all rows) + the consensus",
                                     "ms_per_step": step_s * 1e3}
         print(json.dumps(line), flush=True)
     st.graphs = None

@@ -26,7 +26,17 @@
  *     accepted length out of range, a bounded wait that gave up) are OR-ed into
  *     the caller's int32 `status` word (device pointer, may be NULL) as
  *     ORTHRUS_STATUS_* bits; the affected work is skipped, never trapped.  Read
- *     the word after synchronising the stream.
+ *     the word after synchronising the stream.  The word is passed per call
+ *     rather than kept inside the library (there is no global
+ *     "get status" call): a library-owned word would be shared by every
+ *     stream, thread and CUDA graph of the process, while a caller-owned one
+ *     can be per stream or per step, is captured in graphs like any other
+ *     argument and is cleared by the caller when it chooses.
+ *   - No call takes a host-side context-length hint.  The attention work split
+ *     is computed on the device from ctx_lens, so ctx_lens never has to be
+ *     copied to the host, a whole decode step (attention, consensus, commit)
+ *     runs without a host synchronisation, and a captured graph stays valid as
+ *     the lengths grow.
  *   - Tensors are dense, row-major, with the layouts stated per argument.
  *   - Block slot i of sequence b sits at absolute position ctx_lens[b] + i;
  *     slot 0 is the anchor.
@@ -126,6 +136,14 @@ ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, in
  * Supported: Hq % Hkv == 0; D % 32 == 0, D <= 256; K <= 128; G*K <= 128 for
  * bf16 with D == 128 (tensor-core path); any other accepted shape runs the
  * CUDA-core path.  All pointers 16-byte aligned.
+ *
+ * Residency: the tensor-core path launches one cooperative grid of at most one
+ * CTA per SM whose CTAs merge split partials with each other, so all of them
+ * must run at the same time.  The cooperative launch guarantees that: while
+ * kernels on other streams hold SMs the grid is scheduled only once it fits,
+ * and a device that can never hold it (for example an MPS or green-context
+ * partition with fewer SMs than this device reports) fails the launch with
+ * ORTHRUS_ERR_LAUNCH instead of stalling.
  */
 ORTHRUS_API int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q,
                  const void *k_cache, const void *v_cache,
@@ -238,10 +256,12 @@ ORTHRUS_API int orthrus_attn_path(int B, int Hq, int Hkv, int D, int K, orthrus_
  * about 100 (sequence, KV head) pairs on a 148-SM B200).  The first call on a
  * device looks up the
  * array's device address while that device is current: make it before any
- * stream capture.  All calls share the array, which starts zeroed and is left
- * as orthrus_attn requires of a workspace by every call that completes (a
- * call that timed out may leave it unusable for the rest of the process);
- * calls that overlap on the GPU race.
+ * stream capture.  All calls share the array.  Every call first clears the
+ * array's split-merge counter block on `stream` (an asynchronous memset, no
+ * allocation), so each call starts from the state orthrus_attn requires of a
+ * workspace, even after an earlier call ended with ORTHRUS_STATUS_TIMEOUT.
+ * Calls that overlap on the GPU (other streams, other host threads) race on
+ * the array and must be serialised by the caller.
  */
 #define ORTHRUS_STATIC_SCRATCH_BYTES (16u << 20)
 ORTHRUS_API int orthrus_attn_static(orthrus_view view, orthrus_dtype dtype, const void *q,

@@ -12,11 +12,13 @@
 // every GPU that loads the library holds it until the process exits.  Its
 // device address is looked up once per device, on the first call made while
 // that device is current (cudaGetSymbolAddress), so make the first call on each
-// device before any stream capture.  All calls share the one array; it starts
-// zeroed (a __device__ array is zero-initialised when the module loads), which
-// is what orthrus_attn needs of a fresh workspace, and every completed call
-// leaves its counter block zero again.  Calls that overlap on the GPU (other
-// streams, other host threads) race on the array.
+// device before any stream capture.  All calls share the one array.  Each call
+// first clears the array's split-merge counter block on `stream` (an async
+// memset of a few hundred bytes, no allocation), so a call that gave up on a
+// wait (ORTHRUS_STATUS_TIMEOUT) cannot leave stale counters for the next one;
+// the rest of the array is scratch that every call overwrites before reading.
+// Calls that overlap on the GPU (other streams, other host threads) race on
+// the array.
 #include <mutex>
 
 #include "common.cuh"
@@ -62,6 +64,11 @@ extern "C" int orthrus_attn_static(orthrus_view view, orthrus_dtype dtype, const
     if (need > (size_t)ORTHRUS_STATIC_SCRATCH_BYTES) return ORTHRUS_ERR_WORKSPACE;
     void *scratch = scratch_address();
     if (!scratch) return ORTHRUS_ERR_DEVICE;
+    if (cudaMemsetAsync(scratch, 0, orthrus::kSyncBytes, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return ORTHRUS_ERR_LAUNCH;
+    }
     return orthrus_attn(view, dtype, q, k_cache, v_cache, ctx_lens, B, Hq, Hkv, D, S_max, K,
                         scale, out, scratch, (size_t)ORTHRUS_STATIC_SCRATCH_BYTES, status, stream);
 }

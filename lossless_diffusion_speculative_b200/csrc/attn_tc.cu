@@ -44,6 +44,8 @@
 #include <cudaTypedefs.h>
 #include <stdlib.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -1142,19 +1144,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- host side
 namespace {
 
+// The driver's tensor-map encoder, looked up once per process (thread-safe).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
+    static std::once_flag once;
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    std::call_once(once, [] {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+        else
+            cudaGetLastError();
+    });
     return fn;
 }
 
@@ -1190,27 +1194,33 @@ bool attn_tc_supported(int dtype, int D, int rows)
 
 namespace {
 
-// CTAs of the split for this device, chosen once: one CTA per SM (the
-// kernel's shared memory admits no second one), every CTA resident at once.
+// CTAs of the split for this device, chosen once per device (thread-safe):
+// one CTA per SM (the kernel's shared memory admits no second one).  The
+// launch is cooperative, so all of them are resident at once or the launch
+// fails; the in-kernel split merge relies on that.
+constexpr int kMaxDevices = 64;
+std::once_flag g_ctas_once[kMaxDevices];
+int g_ctas[kMaxDevices];
+
 int resident_ctas()
 {
-    static int ctas[64];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (ctas[dev]) return ctas[dev];
-    int sms = 0, per_sm = 0;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::kSmemAlloc) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::attn_tc_kernel, tc::kThreads,
-                                                      tc::kSmemAlloc) != cudaSuccess ||
-        per_sm < 1) {
-        cudaGetLastError();
-        return 0;
-    }
-    // (capped by the split-merge counter block of the workspace)
-    ctas[dev] = sms * per_sm < kMaxSyncUnits ? sms * per_sm : kMaxSyncUnits;
-    return ctas[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::call_once(g_ctas_once[dev], [dev] {
+        int sms = 0, per_sm = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc::kSmemAlloc) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::attn_tc_kernel, tc::kThreads,
+                                                          tc::kSmemAlloc) != cudaSuccess ||
+            per_sm < 1) {
+            cudaGetLastError();
+            return;
+        }
+        // (capped by the split-merge counter block of the workspace)
+        g_ctas[dev] = sms * per_sm < kMaxSyncUnits ? sms * per_sm : kMaxSyncUnits;
+    });
+    return g_ctas[dev];
 }
 
 }  // namespace
@@ -1242,11 +1252,16 @@ cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st)
     cfg.blockDim = dim3(tc::kThreads);
     cfg.dynamicSmemBytes = tc::kSmemAlloc;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    // cooperative: every CTA is resident at once (the split merge waits on
+    // sibling CTAs), or the launch fails; programmatic dependent launch lets
+    // the prologue overlap the previous kernel in the stream
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tk, tv, p);
 }
 

@@ -105,7 +105,7 @@ class DecodeStep:
         ob.orthrus_kv_commit(self.ctx, self.accepted, K=w.K, Hkv=w.Hkv, D=w.D, S_max=w.S_max,
                              dtype=self.dtype, num_layers=self.L, status=self.status)
 
-    def segments(self, chunk: int = 0):
+    def segments(self, chunk: int = 0, order: Optional[str] = None):
         """The step as ordered launch segments (timed separately by the bench).
 
         With ``chunk`` > 0 (cold order) each view runs as layer groups of that
@@ -113,7 +113,8 @@ class DecodeStep:
         smaller segments, so that a caller feeding the step from the host can
         start each group once its inputs have arrived.
         """
-        if self.order == "cold" and chunk > 0:
+        order = self.order if order is None else order
+        if order == "cold" and chunk > 0:
             segs = []
             for view, vn in ((ob.DIFF, "diff"), (ob.AR, "ar")):
                 for c in range(0, self.L, chunk):
@@ -122,7 +123,7 @@ class DecodeStep:
                     segs.append((f"attn_{vn}_{c}", lambda v=view, ls=layers: [self._attn(v, l) for l in ls]))
             segs.append(("consensus_commit", self._tail))
             return segs
-        if self.order == "cold":
+        if order == "cold":
             return [("write_block_diff", lambda: self._write_block(ob.DIFF)),
                     ("attn_diff", lambda: self._attn_view(ob.DIFF)),
                     ("write_block_ar", lambda: self._write_block(ob.AR)),
@@ -146,9 +147,11 @@ class DecodeStep:
         for _, fn in self.segments(chunk):
             fn()
 
-    def capture(self, stream: torch.cuda.Stream, chunk: int = 0):
+    def capture(self, stream: torch.cuda.Stream, chunk: int = 0, order: Optional[str] = None):
         """CUDA graphs of the reset and of every segment (captured on ``stream``)."""
-        self.run_eager(chunk)               # warm: attributes set, plans cached
+        self.reset()
+        for _, fn in self.segments(chunk, order):   # warm: attributes set, plans cached
+            fn()
         torch.cuda.synchronize()
         graphs = []
         with torch.cuda.stream(stream):
@@ -156,7 +159,7 @@ class DecodeStep:
             with torch.cuda.graph(g, stream=stream):
                 self.reset()
             graphs.append(("reset", g))
-            for name, fn in self.segments(chunk):
+            for name, fn in self.segments(chunk, order):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
                     fn()
@@ -174,6 +177,10 @@ class DecodeStep:
         """Verified tokens one step commits: sum_b min(a_b + 1, K) (planted a)."""
         a = self.consensus_in.planted_accept
         return int(np.minimum(a + 1, self.w.K).sum())
+
+    def tokens_per_step_expected(self) -> float:
+        """The same count's expectation under the workload's acceptance law."""
+        return wl.expected_tokens_per_step(self.w)
 
     def kv_bytes_per_attn_call(self) -> int:
         return self.w.kv_bytes_per_view_layer()

@@ -228,6 +228,32 @@ def planted_accept_lengths(w: Workload) -> np.ndarray:
     return np.minimum(a, w.K).astype(np.int32)
 
 
+def expected_tokens_per_step(w: Workload) -> float:
+    """E[sum_b min(a_b + 1, K)] under the workload's planted acceptance law
+    (the seeded draw gives one sample of it; the kernels' time does not depend
+    on it).  Per sequence:
+      fixed:a   min(a + 1, K)
+      geom:p    a = min(X - 1, K), X ~ Geometric(p) on {1, 2, ...}:
+                E[min(X, K)] = sum_{j=1..K} P(X >= j) = (1 - (1 - p)^K) / p
+      uniform   a ~ U{0..K}: (sum_{a<K} (a + 1) + K) / (K + 1)
+      half      a = K // 2: min(K // 2 + 1, K)
+    """
+    K = w.K
+    kind, _, arg = w.plant.partition(":")
+    if kind == "fixed":
+        per = min(int(arg) + 1, K)
+    elif kind == "geom":
+        p = float(arg)
+        per = (1.0 - (1.0 - p) ** K) / p
+    elif kind == "uniform":
+        per = (K * (K + 1) / 2 + K) / (K + 1)
+    elif kind == "half":
+        per = min(K // 2 + 1, K)
+    else:
+        raise ValueError(w.plant)
+    return float(w.B * per)
+
+
 def consensus_inputs(w: Workload, accept: Optional[np.ndarray] = None,
                      B: Optional[int] = None) -> ConsensusInputs:
     """Logits ~ N(0, sigma) with a planted unique argmax per row (margin 1.0)

@@ -47,17 +47,3 @@ def assert_attn_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
     err = float(np.max(np.abs(got - ref)))
     assert err <= ATOL_REL_RMS * rms, f"{what}: max|err| {err:.3e} > {ATOL_REL_RMS} * rms {rms:.3e}"
     return err / rms
-
-
-def sample_rows(B, K, Hq, n, seed, ctx=None):
-    """(b, i, h) triples: edge slots (0, K-1), every sequence and head group
-    boundary, plus a seeded random sample."""
-    rng = np.random.default_rng(seed)
-    rows = set()
-    for b in range(B):
-        for i in {0, K - 1, K // 2}:
-            for h in {0, Hq - 1}:
-                rows.add((b, i, h))
-    while len(rows) < n:
-        rows.add((int(rng.integers(B)), int(rng.integers(K)), int(rng.integers(Hq))))
-    return np.array(sorted(rows), dtype=np.int32)

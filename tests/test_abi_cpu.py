@@ -78,3 +78,17 @@ def test_host_checks_reject_bad_arguments_without_a_device(lib):
                                  8, 0, None, None) == binding.ERR_UNSUPPORTED
     assert lib.orthrus_kv_commit(1, None, None, None, None, None, vp(16), 1, 8, 128, 64, 8, 0,
                                  None, None) == binding.ERR_ARG
+
+
+def test_device_status_is_a_per_call_word():
+    """Every entry point that enqueues device work takes the caller's status
+    word; the library keeps no global status (there is no get-status call),
+    and no entry point takes a host-side context-length hint (the work split
+    is computed on the device from ctx_lens)."""
+    src = open(os.path.join(ROOT, "include", "orthrus.h")).read()
+    decls = dict(re.findall(r"ORTHRUS_API\s+[\w\s\*]*?\b(orthrus_\w+)\s*\(([^;]*)\);", src))
+    for name in ("orthrus_attn", "orthrus_attn_static", "orthrus_consensus",
+                 "orthrus_kv_commit", "orthrus_write_block"):
+        assert re.search(r"int32_t\s*\*\s*status", decls[name]), name
+        assert "hint" not in decls[name], name
+    assert not any("status" in n for n in decls), sorted(decls)

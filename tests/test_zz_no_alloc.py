@@ -2,8 +2,9 @@
 memory (an engine whose memory plan is frozen after warm-up, a plugin that only
 receives input and output pointers, a runtime whose allocator belongs to
 another framework).  It uses the library's built-in scratch array instead of a
-caller workspace; its results must match orthrus_attn's on consecutive calls
-(the shared scratch keeps the previous call's contents).
+caller workspace; its results must match the fp64 oracle and orthrus_attn's on
+consecutive calls (the shared scratch keeps the previous call's contents), and
+warm calls must not change the device's free memory.
 
 This file is collected last on purpose."""
 import ctypes
@@ -12,7 +13,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from lossless_diffusion_speculative_b200 import binding as ob
+from lossless_diffusion_speculative_b200 import workloads as wl
 from gpu_util import assert_attn_close, run_attn, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -43,14 +46,21 @@ def _call_static(view, q, kc, vc, ctx, dtype_code):
     return out
 
 
-def _inputs(seed, B, Hq, Hkv, D, K, ctx, dtype):
+def _host_inputs(seed, B, Hq, Hkv, D, K, ctx, dtype):
+    """Seeded inputs as float32 arrays holding exactly the values uploaded."""
     rng = np.random.default_rng(seed)
     ctx = np.asarray(ctx, np.int32)
     S = int(ctx.max()) + K
     sc = np.float32(1 / np.sqrt(128))
-    q = rng.standard_normal((B, K, Hq, D), dtype=np.float32) * sc
-    kc = rng.standard_normal((B, Hkv, S, D), dtype=np.float32) * sc
-    vc = rng.standard_normal((B, Hkv, S, D), dtype=np.float32) * sc
+    f = wl.round_to_bf16 if dtype == torch.bfloat16 else (lambda x: x)
+    q = f(rng.standard_normal((B, K, Hq, D), dtype=np.float32) * sc)
+    kc = f(rng.standard_normal((B, Hkv, S, D), dtype=np.float32) * sc)
+    vc = f(rng.standard_normal((B, Hkv, S, D), dtype=np.float32) * sc)
+    return q, kc, vc, ctx
+
+
+def _inputs(seed, B, Hq, Hkv, D, K, ctx, dtype):
+    q, kc, vc, ctx = _host_inputs(seed, B, Hq, Hkv, D, K, ctx, dtype)
     return (to_dev(q, dtype), to_dev(kc, dtype), to_dev(vc, dtype),
             torch.from_numpy(ctx).cuda())
 
@@ -64,12 +74,34 @@ SHAPES = {   # (B, Hq, Hkv, D, K, ctx) of two consecutive calls
 @pytest.mark.parametrize("name,dtype,code", [("bf16_tensor_core", torch.bfloat16, ob.BF16),
                                              ("f32_cuda_core", torch.float32, ob.F32)])
 def test_static_scratch_matches_workspace_call_twice(name, dtype, code):
-    cases = [(view, _inputs(10 + view, *shape, dtype))      # two calls in a row
+    cases = [(view, shape, _inputs(10 + view, *shape, dtype))      # two calls in a row
              for view, shape in zip((ob.DIFF, ob.AR), SHAPES[name])]
-    for view, (q, kc, vc, ctx) in cases:
-        got = _call_static(view, q, kc, vc, ctx, code)
+    for view, shape, (q, kc, vc, ctx) in cases:
+        got = _call_static(view, q, kc, vc, ctx, code).cpu().numpy()
         ref = run_attn(view, q, kc, vc, ctx, dtype)
-        assert_attn_close(got.cpu().numpy(), ref.cpu().numpy(), "static scratch")
+        assert_attn_close(got, ref.cpu().numpy(), "static scratch vs orthrus_attn")
+        hq, hk, hv, hc = _host_inputs(10 + view, *shape, dtype)
+        assert_attn_close(got, oracle.attention(view, hq, hk, hv, hc), "static scratch vs oracle")
+
+
+def test_static_scratch_calls_allocate_nothing():
+    """After a warm call (which loads the library's device code, scratch array
+    included), further calls leave the device's free memory unchanged."""
+    q, kc, vc, ctx = _inputs(21, 2, 32, 8, 128, 32, [5000, 300], torch.bfloat16)
+    _call_static(ob.DIFF, q, kc, vc, ctx, ob.BF16)
+    B, K, Hq, D = q.shape
+    out = torch.empty((B, K, Hq, D), dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    f = _static_fn()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for rep in range(6):
+        rc = f(rep % 2, ob.BF16, q.data_ptr(), kc.data_ptr(), vc.data_ptr(), ctx.data_ptr(),
+               B, Hq, 8, D, kc.shape[2], K, 0.0, out.data_ptr(), None, stream)
+        assert rc == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
 
 
 def test_static_scratch_rejects_oversized_problems():
