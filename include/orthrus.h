@@ -89,7 +89,7 @@ typedef enum {
 
 /*
  * orthrus_attn_workspace_size — bytes of scratch orthrus_attn needs for these
- * sizes on the CURRENT device (a 1280-byte block of split-merge counters, then
+ * sizes on the CURRENT device (a 1920-byte block of split-merge flags and counters, then
  * the split-KV partials: one fp32 [G*K, D] tile plus G*K log-sum-exp values
  * per (split unit, KV segment) boundary).  Independent of the context
  * lengths.  Returns 0 for invalid sizes.

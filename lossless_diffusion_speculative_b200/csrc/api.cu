@@ -109,6 +109,8 @@ int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const vo
     if (!attn_shape_ok(B, Hq, Hkv, D, S_max, K, dtype)) return ORTHRUS_ERR_ARG;
     if (K > S_max) return ORTHRUS_ERR_ARG;
     if (!(scale == scale) || isinf(scale)) return ORTHRUS_ERR_ARG;
+    // the on-device work split counts 64-key boxes over all segments in 32 bits
+    if ((int64_t)B * Hkv * ((S_max + 63) / 64) >= (int64_t)1 << 31) return ORTHRUS_ERR_UNSUPPORTED;
     if (!attn_shape_supported(Hq, Hkv, D, K)) return ORTHRUS_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (workspace && !aligned16(workspace)))
@@ -128,8 +130,9 @@ int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const vo
     a.out = out;
     char *ws = static_cast<char *>(workspace);
     a.ws_sync = reinterpret_cast<int32_t *>(ws);
-    a.ws_o = reinterpret_cast<float *>(ws + kSyncBytes);
-    a.ws_lse = reinterpret_cast<float *>(ws + kSyncBytes + attn_ws_o_bytes(pl.slots, rows, D));
+    a.ws_plan = reinterpret_cast<int32_t *>(ws + kSyncBytes);
+    a.ws_o = reinterpret_cast<float *>(ws + kSyncBytes + kPlanBytes);
+    a.ws_lse = reinterpret_cast<float *>(ws + kSyncBytes + kPlanBytes + attn_ws_o_bytes(pl.slots, rows, D));
     a.status = status;
     a.B = B;
     a.Hq = Hq;

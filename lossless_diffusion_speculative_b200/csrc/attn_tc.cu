@@ -76,11 +76,10 @@ constexpr uint32_t kSmemStage = kSmemK;
 static_assert(kSmemStage + kRows * kStagePitch * 4 <= kSmemBar, "staging rows fit in the rings");
 // split merge, after the last piece, over the idle query tile and rings: the
 // gathered partial rows (n x nr rows of D floats, n * nr < rows + n <= 128 +
-// kMaxSyncUnits), their log2-sum-exp rows (n x nl floats, nl <= nr + 6) and
+// kMaxSyncUnits), their log2-sum-exp runs (n x nl floats, nl <= nr + 6) and
 // two weight rows per warp (8 x n floats)
 constexpr uint32_t kSmemGather = kSmemQ;
-constexpr int kLseOneCopy = 16384;                      // bytes: the lse rows of all partials in one copy
-static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + kLseOneCopy + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
+static_assert(kSmemGather + (kRows + kMaxSyncUnits) * kD * 4 + (kRows + 7 * kMaxSyncUnits) * 4 + 16 +
                       8 * kMaxSyncUnits * 4 <= kSmemBar,
               "split merge fits in the rings");
 
@@ -104,9 +103,11 @@ enum : int {
 };
 
 constexpr uint32_t kSmemMisc = kSmemBar + B_COUNT * 8;
-// (after tmem address and abort flag) the split (W, P) and 2 shared pieces
-constexpr uint32_t kSmemPend = kSmemMisc + 16;
-constexpr uint32_t kSmemUsed = kSmemPend + 16 + 2 * 32;
+// (after tmem address and abort flag) the CTA's work plan, then the (at most
+// two) pieces of its range whose segments other CTAs share
+constexpr uint32_t kSmemPlan = kSmemMisc + 16;
+constexpr uint32_t kSmemPend = kSmemPlan + 48;
+constexpr uint32_t kSmemUsed = kSmemPend + 2 * 32;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;       // room to align the base to 1 KiB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = kSBuf * 128;                 // 384: O accumulator
@@ -397,6 +398,13 @@ __device__ __forceinline__ int32_t counter_load_acquire(const int32_t *c)
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
     return v;
 }
+__device__ __forceinline__ int32_t counter_load_relaxed(const int32_t *c)
+{
+    int32_t v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ int32_t counter_fetch_add_acq_rel(int32_t *c, int32_t v)
 {
     int32_t old;
@@ -418,6 +426,230 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major)
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+
+// ---------------------------------------------------------------- work split
+// The key space of every (sequence b, KV head g) segment, len_b = ctx_b + K
+// keys (0 when ctx_b is out of range), is counted in 64-key boxes, nbx_b =
+// ceil(len_b / 64) per segment; all segments are laid end to end in the order
+// s = b * Hkv + g and the flat box space [0, NB) is cut into P equal ranges
+// (to a box), one per CTA.  A range meets one or more segments; each meeting
+// is a piece.  Pieces start on a box boundary of their segment and end on one
+// or at the segment's end, so only a segment's last box is ever partial.  In
+// every (CTA c, segment s) piece the CTA writes the final rows when it covers
+// s alone, else a partial in workspace slot c + s (unique: consecutive CTAs
+// share at most one segment).  All of it is 32-bit arithmetic (the host keeps
+// B * Hkv * ceil(S_max / 64) below 2^31).
+struct Plan {
+    int NB;          // boxes over all segments
+    int P;           // CTAs with work (P <= grid)
+    int q, r;        // NB = q * P + r (range starts: c * q + c * r / P)
+    int lo, hi;      // this CTA's box range [lo, hi)
+    int b0;          // first sequence whose segments meet the range (B: none)
+    int off0;        // flat box offset of sequence b0
+    int g0;          // KV head of the range's first piece
+    int len0;        // length of sequence b0's segments
+};
+static_assert(sizeof(Plan) == 40, "plan slot");
+
+__device__ __forceinline__ int nbox_of(int len) { return (len + kBoxKeys - 1) / kBoxKeys; }
+
+__device__ __forceinline__ int plan_start(const Plan &pl, int c) { return c * pl.q + (c * pl.r) / pl.P; }
+
+// The CTA whose range holds flat box x: max{c : plan_start(c) <= x}.
+__device__ __forceinline__ int plan_cta_of(const Plan &pl, int x)
+{
+    return (int)(((int64_t)(x + 1) * pl.P - 1) / pl.NB);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+struct PlanArgs {
+    const int32_t *ctx_lens;
+    int32_t *status;
+    int B, Hkv, K, S_max;
+};
+
+// Computed by all 32 lanes of one warp (lane l reads ctx_lens[l], [l + 32],
+// ...); every lane returns the same plan.  CTA 0 also raises
+// ORTHRUS_STATUS_CAPACITY for every sequence without room for its block.
+__device__ __noinline__ Plan make_plan(const PlanArgs p, int grid, int cid, int min_boxes)
+{
+    const int lane = threadIdx.x & 31;
+    Plan pl;
+    int NB = 0, len_first = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        int len = 0;
+        if (b < p.B) {
+            len = seg_len(p.ctx_lens, b, p.K, p.S_max);
+            if (len == 0 && cid == 0) raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
+        }
+        if (base == 0) len_first = len;
+        NB += __shfl_sync(0xffffffffu, warp_incl_scan(p.Hkv * nbox_of(len), lane), 31);
+    }
+    pl.NB = NB;
+    int P = NB > 0 ? (NB + min_boxes - 1) / min_boxes : 1;
+    if (P > grid) P = grid;
+    pl.P = P;
+    pl.q = NB / P;
+    pl.r = NB - pl.q * P;
+    pl.lo = plan_start(pl, cid);
+    pl.hi = plan_start(pl, cid + 1);
+    pl.b0 = p.B;
+    pl.off0 = 0;
+    pl.g0 = 0;
+    pl.len0 = 0;
+    if (cid < P && pl.hi > pl.lo) {
+        int carry = 0;
+        for (int base = 0; base < p.B; base += 32) {
+            const int b = base + lane;
+            int len = len_first;
+            if (base > 0) len = b < p.B ? seg_len(p.ctx_lens, b, p.K, p.S_max) : 0;
+            const int nb = p.Hkv * nbox_of(len);
+            const int incl = warp_incl_scan(nb, lane);
+            const int start = carry + incl - nb;
+            const unsigned hit = __ballot_sync(0xffffffffu, nb > 0 && start <= pl.lo && pl.lo < start + nb);
+            if (hit) {
+                const int l = __ffs(hit) - 1;
+                pl.b0 = base + l;
+                pl.off0 = __shfl_sync(0xffffffffu, start, l);
+                pl.len0 = __shfl_sync(0xffffffffu, len, l);
+                pl.g0 = (pl.lo - pl.off0) / nbox_of(pl.len0);
+                break;
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    return pl;
+}
+
+// Cached plans (in the workspace): entry c, for CTA c, holds
+//   [0] tag, [1] B, [2] Hkv, [3] K, [4] S_max, [5] grid, [6] min_boxes, [7] 0,
+//   [8, 8 + B) the ctx_lens values the plan was computed for, [40, 50) the plan.
+// Each CTA reads and writes only its own entry; a later call sees what an
+// earlier one wrote (griddepcontrol.wait / stream order).
+constexpr int kPlanTag = 0x4F525448;
+constexpr int kPlanAt = 40;
+static_assert(kPlanAt + 10 <= kPlanEntryInts && 8 + kPlanMaxB <= kPlanAt, "plan entry layout");
+
+// The CTA's plan, by all 32 lanes of one warp: the cached entry when its key
+// and lengths match the live ones (one round of loads), else computed and
+// cached.  Lane 0 stores it to *out.
+__device__ __noinline__ void plan_prologue(const PlanArgs p, int32_t *cache, int grid, int cid,
+                                           int min_boxes, Plan *out)
+{
+    const int lane = threadIdx.x & 31;
+    int32_t *e = cache + (size_t)cid * kPlanEntryInts;
+    if (p.B <= kPlanMaxB) {
+        // ints [0, 52) of the entry, 16 bytes per lane, and the live lengths
+        int4 w = make_int4(0, 0, 0, 0);
+        if (lane < 13) w = *reinterpret_cast<const int4 *>(e + 4 * lane);
+        const int live = lane < p.B ? __ldg(p.ctx_lens + lane) : 0;
+        const int src = 2 + (lane >> 2), comp = lane & 3;      // cached length of sequence `lane`
+        const int cx = __shfl_sync(0xffffffffu, w.x, src), cy = __shfl_sync(0xffffffffu, w.y, src);
+        const int cz = __shfl_sync(0xffffffffu, w.z, src), cw = __shfl_sync(0xffffffffu, w.w, src);
+        const int cached = comp == 0 ? cx : comp == 1 ? cy : comp == 2 ? cz : cw;
+        bool bad = lane < p.B && cached != live;
+        if (lane == 0) bad |= w.x != kPlanTag || w.y != p.B || w.z != p.Hkv || w.w != p.K;
+        if (lane == 1) bad |= w.x != p.S_max || w.y != grid || w.z != min_boxes;
+        if (!__any_sync(0xffffffffu, bad)) {
+            // hit: the plan is ints [40, 50): lanes 10, 11 and 12
+            int v[12];
+            const int4 a = make_int4(__shfl_sync(0xffffffffu, w.x, 10), __shfl_sync(0xffffffffu, w.y, 10),
+                                     __shfl_sync(0xffffffffu, w.z, 10), __shfl_sync(0xffffffffu, w.w, 10));
+            const int4 b = make_int4(__shfl_sync(0xffffffffu, w.x, 11), __shfl_sync(0xffffffffu, w.y, 11),
+                                     __shfl_sync(0xffffffffu, w.z, 11), __shfl_sync(0xffffffffu, w.w, 11));
+            const int c0 = __shfl_sync(0xffffffffu, w.x, 12), c1 = __shfl_sync(0xffffffffu, w.y, 12);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            v[8] = c0; v[9] = c1;
+            if (lane == 0) {
+                Plan pl;
+                pl.NB = v[0]; pl.P = v[1]; pl.q = v[2]; pl.r = v[3]; pl.lo = v[4]; pl.hi = v[5];
+                pl.b0 = v[6]; pl.off0 = v[7]; pl.g0 = v[8]; pl.len0 = v[9];
+                *out = pl;
+            }
+            // (capacity errors are raised again on every call, not cached)
+            if (cid == 0 && lane < p.B && seg_len(p.ctx_lens, lane, p.K, p.S_max) == 0)
+                raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
+            return;
+        }
+    }
+    const Plan pl = make_plan(p, grid, cid, min_boxes);
+    if (lane == 0) *out = pl;
+    if (p.B <= kPlanMaxB) {
+        if (lane < p.B) e[8 + lane] = __ldg(p.ctx_lens + lane);
+        if (lane == 0) {
+            *reinterpret_cast<int4 *>(e) = make_int4(kPlanTag, p.B, p.Hkv, p.K);
+            *reinterpret_cast<int4 *>(e + 4) = make_int4(p.S_max, grid, min_boxes, 0);
+            *reinterpret_cast<int4 *>(e + kPlanAt) = make_int4(pl.NB, pl.P, pl.q, pl.r);
+            *reinterpret_cast<int4 *>(e + kPlanAt + 4) = make_int4(pl.lo, pl.hi, pl.b0, pl.off0);
+            *reinterpret_cast<int2 *>(e + kPlanAt + 8) = make_int2(pl.g0, pl.len0);
+        }
+    }
+}
+
+// One piece: segment (b, g) meets the CTA's range in keys [a, e).
+struct TPiece {
+    int b, g, s;     // sequence, KV head, segment index b * Hkv + g
+    int len;         // segment length in keys
+    int a, e;        // keys [a, e) of the segment, 0 <= a < e <= len, a a multiple of 64
+    int s0, nbx;     // flat box start of the segment, its box count
+};
+
+// Iterates the pieces of the CTA's range in flat order (from the plan).
+struct BoxIter {
+    const int32_t *ctx;
+    int B, Hkv, K, S_max;
+    int lo, hi, b, g, off, nbx, len;
+
+    __device__ __forceinline__ BoxIter(const Plan &pl, const AttnArgs &p)
+        : ctx(p.ctx_lens), B(p.B), Hkv(p.Hkv), K(p.K), S_max(p.S_max), lo(pl.lo), hi(pl.hi), b(pl.b0),
+          g(pl.g0), off(pl.off0), nbx(nbox_of(pl.len0)), len(pl.len0)
+    {
+    }
+
+    __device__ __forceinline__ bool next(TPiece &pc)
+    {
+        while (b < B) {
+            if (nbx == 0 || g >= Hkv) {
+                off += Hkv * nbx;
+                ++b;
+                g = 0;
+                len = b < B ? seg_len(ctx, b, K, S_max) : 0;
+                nbx = nbox_of(len);
+                continue;
+            }
+            const int s0 = off + g * nbx;
+            if (s0 >= hi) return false;
+            const int A = lo > s0 ? lo : s0, E = hi < s0 + nbx ? hi : s0 + nbx;
+            pc.b = b;
+            pc.g = g;
+            pc.s = b * Hkv + g;
+            pc.len = len;
+            pc.s0 = s0;
+            pc.nbx = nbx;
+            pc.a = (A - s0) * kBoxKeys;
+            pc.e = (E - s0) * kBoxKeys < len ? (E - s0) * kBoxKeys : len;
+            ++g;
+            if (E > A) return true;
+        }
+        return false;
+    }
+};
+
+// The same, not inlined: the softmax warps' iterator then lives in local
+// memory (touched once per piece) instead of holding registers through the
+// tile loop, where the softmax needs every register it can get.
+__device__ __noinline__ bool next_piece(BoxIter &it, TPiece &pc) { return it.next(pc); }
 
 // ---------------------------------------------------------------- tiling
 // A piece [a, e) is read in 64-key boxes; box k starts at a + 64k except the
@@ -442,15 +674,20 @@ struct Tiling {
 };
 
 // A segment shared with other CTAs: the n CTAs [c_lo, c_lo + n) hold its
-// partials in workspace slots c_lo + s, ..., c_lo + n - 1 + s.
+// partials in workspace slots c_lo + s, ..., c_lo + n - 1 + s.  The segment
+// is the last piece of every one of them except the last CTA, c_lo + n - 1,
+// for which it is the first piece; it is also that CTA's last piece when
+// hi_last (its range ends within the segment).
 struct SplitInfo {
     int b, g, s, c_lo, n;
+    bool hi_last;
 };
 // What the epilogue records of a shared piece (in shared memory, so that
 // nothing stays live in registers across the tile loop).
 struct SharedPiece {
-    int64_t s0;
-    int b, g, s, len;
+    int s0, nbx;     // flat box start and box count of the segment
+    int b, g, s;
+    int idx;         // position of the piece in the CTA's range
 };
 
 struct Shared {
@@ -469,14 +706,14 @@ struct Shared {
 // tiles into the V ring.  Each ring is filled as soon as it has a free slot (K
 // before V when both have), so a V tile never waits for a K slot or the other
 // way round.
-__device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                         int cid, const CUtensorMap *tq, const CUtensorMap *tk,
+__device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, const Plan &pl,
+                                         const CUtensorMap *tq, const CUtensorMap *tk,
                                          const CUtensorMap *tv)
 {
     const int G = p.Hq / p.Hkv;
     const uint32_t q_bytes = 2u * 128u * G * p.K;
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
-    Piece pc;
+    BoxIter it(pl, p);
+    TPiece pc;
     uint32_t piece = 0, qloads = 0, kq = 0, kv = 0;   // pieces, Q tiles, K tiles, V tiles
     bool ok = true;
     auto slot_free = [&](uint32_t item, int nst, int bempty) {
@@ -575,11 +812,11 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
 //   PV thread: O += P(t) V(t) once P(t) is written and V(t) has landed (the
 //              first PV of a piece also waits until the previous piece's O
 //              has been read out)
-__device__ __forceinline__ void s_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                         int cid, uint32_t tmem)
+__device__ __forceinline__ void s_issuer(const Shared &sh, const AttnArgs &p, const Plan &pl,
+                                         uint32_t tmem)
 {
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
-    Piece pc;
+    BoxIter it(pl, p);
+    TPiece pc;
     uint32_t qp = 0, kq = 0, gt = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
@@ -614,12 +851,12 @@ __device__ __forceinline__ void s_issuer(const Shared &sh, const AttnArgs &p, co
     }
 }
 
-__device__ __forceinline__ void pv_issuer(const Shared &sh, const AttnArgs &p, const Decomp &d,
-                                          int cid, uint32_t tmem)
+__device__ __forceinline__ void pv_issuer(const Shared &sh, const AttnArgs &p, const Plan &pl,
+                                          uint32_t tmem)
 {
     const uint32_t idesc_pv = instr_desc(128, 128, true);
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
-    Piece pc;
+    BoxIter it(pl, p);
+    TPiece pc;
     uint32_t qp = 0, kv = 0, gt = 0;
     bool ok = true;
     while (ok && it.next(pc)) {
@@ -707,14 +944,18 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&s)[128], int nb, float 
     return lsum.x + lsum.y;
 }
 
-// Merge of one shared segment, by CTA cid (see softmax_epilogue).  Thread 0
-// waits until all n CTAs have published; warp 0 then gathers this CTA's share
-// of the rows of all n partials, with their log2-sum-exp values, into shared
-// memory (lane q issues the bulk copies of partial q), and thread 0 leaves
-// (depart[c_lo] += 1; the last to leave resets both counters).  Each warp then
-// merges whole rows, two at a time: lanes compute the weights 2^(lse_q - max)
-// / sum of the rows' partials (the log-sum-exp merge of flash-decoding), then
-// lane c4 accumulates 16-byte column c4 over the partials and stores it.
+// Merge of one shared segment, by CTA cid (see softmax_epilogue).  Every
+// partial is published by its row-warps (flag += 1 each, release).  Lane q of
+// warp 0 watches the flag of the segment's CTA c_lo + q and, once it is
+// complete, gathers that partial's share of rows for this CTA (nr rows from
+// r_lo, stored with the 16-byte-chunk swizzle of the epilogue) and their
+// log2-sum-exp values into shared memory with bulk copies, so the gather
+// overlaps the wait for the segment's slowest CTA.  Once every flag has been
+// seen the CTA departs (depart[c_lo] += 1; the last to depart clears the
+// segment's flags and the counter for the next call).  Each warp then merges
+// whole rows, two at a time: lanes compute the weights 2^(lse_q - max) / sum
+// of the rows' partials (the log-sum-exp merge of flash-decoding), then lane
+// c4 accumulates 16-byte column c4 over the partials and stores it.
 // Returns the B_GATHER phases used (0 or 1), or -1 after an abort.
 __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag, uint8_t *smem,
                                         int32_t *ws_sync, const float *ws_o, const float *ws_lse,
@@ -726,52 +967,61 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
     const int lp = lse_pitch(rows);
     const int j = cid - sp.c_lo;
     const int r_lo = j * rows / sp.n, nr = (j + 1) * rows / sp.n - r_lo;
-    // log2-sum-exp values: when the n partials' whole lse rows are small
-    // (n * lp floats, contiguous in the workspace) one bulk copy brings them
-    // all, else each partial's 16-byte-aligned run covering this CTA's rows
-    const bool one_lse = sp.n * lp * 4 <= kLseOneCopy;
-    const int l_lo = one_lse ? 0 : r_lo & ~3;
-    const int nl = one_lse ? lp : ((r_lo + nr + 3) & ~3) - l_lo;     // lse floats per partial
+    // each partial's log2-sum-exp run covering this CTA's rows, 16-byte aligned
+    const int l_lo = r_lo & ~3;
+    const int nl = ((r_lo + nr + 3) & ~3) - l_lo;                       // lse floats per partial
     const uint32_t o_bytes = (uint32_t)nr * kD * 4, l_bytes = (uint32_t)nl * 4;
     const uint32_t s_lse = kSmemGather + (uint32_t)sp.n * o_bytes;     // after the O rows
     const uint32_t s_w = s_lse + (((uint32_t)sp.n * l_bytes + 15u) & ~15u);   // [4 warps][2][n] weights
-    int32_t *arrive = ws_sync + sp.c_lo;
+    const int c_hi = sp.c_lo + sp.n - 1;
+    const int nw = (rows + 31) >> 5;                                    // row-warps per partial
+    // the flag CTA c of the segment sets: its last piece's, except for c_hi
+    // when the segment is its first piece but not its last
+    auto flag_of = [&](int c) {
+        return ws_sync + ((c == c_hi && !sp.hi_last) ? kSyncFirst : kSyncLast) * kMaxSyncUnits + c;
+    };
+    bool ok = true;
     if (warp == 0) {
-        bool ok = true;
-        if (lane == 0) {
-            const unsigned long long t0 = global_ns();
-            while (counter_load_acquire(arrive) < sp.n) {
-                if (*abort_flag || global_ns() - t0 > kTimeoutNs) {
-                    *abort_flag = 1;
-                    raise_status(status, ORTHRUS_STATUS_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok && nr > 0) mbar_expect_tx(bar, (uint32_t)sp.n * (o_bytes + l_bytes));
-        }
-        if (!__shfl_sync(0xffffffffu, ok, 0)) return -1;
-        // (lane 0's acquire covers the warp: __syncwarp orders the lanes after
-        // it, and the proxy fence orders the bulk reads after both)
-        __syncwarp();
-        fence_proxy_async_global();
         if (nr > 0) {
+            if (lane == 0) mbar_expect_tx(bar, (uint32_t)sp.n * (o_bytes + l_bytes));
+            __syncwarp();
             for (int q = lane; q < sp.n; q += 32) {
+                const int32_t *flag = flag_of(sp.c_lo + q);
+                if (counter_load_relaxed(flag) < nw) {
+                    const unsigned long long t0 = global_ns();
+                    while (counter_load_relaxed(flag) < nw) {
+                        if (*abort_flag || global_ns() - t0 > kTimeoutNs) {
+                            *abort_flag = 1;
+                            raise_status(status, ORTHRUS_STATUS_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+                if (!ok) break;
+                // (the fence after the relaxed read that saw the releases orders
+                // the partial's writes before this lane's later reads; the
+                // proxy fence extends that to its bulk reads)
+                fence_acquire_gpu();
+                fence_proxy_async_global();
                 const size_t slot = (size_t)sp.c_lo + q + sp.s;
                 bulk_load(base + kSmemGather + q * o_bytes, ws_o + (slot * rows + r_lo) * kD, o_bytes, bar);
-                if (!one_lse) bulk_load(base + s_lse + q * l_bytes, ws_lse + slot * lp + l_lo, l_bytes, bar);
+                bulk_load(base + s_lse + q * l_bytes, ws_lse + slot * lp + l_lo, l_bytes, bar);
             }
-            if (one_lse && lane == 0)
-                bulk_load(base + s_lse, ws_lse + ((size_t)sp.c_lo + sp.s) * lp, (uint32_t)sp.n * l_bytes, bar);
         }
-        if (lane == 0 && counter_fetch_add_acq_rel(ws_sync + kMaxSyncUnits + sp.c_lo, 1) == sp.n - 1) {
-            arrive[0] = 0;                                    // everyone has passed the wait
-            ws_sync[kMaxSyncUnits + sp.c_lo] = 0;
+        ok = __all_sync(0xffffffffu, ok);
+        // every lane has seen its flags: depart; the last CTA to leave clears them
+        int last = 0;
+        if (ok && lane == 0)
+            last = counter_fetch_add_acq_rel(ws_sync + kSyncDepart * kMaxSyncUnits + sp.c_lo, 1) == sp.n - 1;
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+            for (int q = lane; q < sp.n; q += 32) *flag_of(sp.c_lo + q) = 0;
+            if (lane == 0) ws_sync[kSyncDepart * kMaxSyncUnits + sp.c_lo] = 0;
         }
     }
-    if (nr == 0) return 0;
-    if (!wait_bar(bar, gph & 1, abort_flag, status)) {
-        if (warp == 0) wait_bar_quiet(bar, gph & 1);          // let the copies land
+    if (nr == 0) return ok ? 0 : -1;
+    if (!ok || !wait_bar(bar, gph & 1, abort_flag, status)) {
+        if (warp == 0) wait_bar_quiet(bar, gph & 1);          // let the copies issued land
         return -1;
     }
     const float4 *gbuf = reinterpret_cast<const float4 *>(smem + kSmemGather);
@@ -809,8 +1059,10 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
         const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
         float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
         float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
-        const float4 *v = gbuf + r * 32 + lane, *u = gbuf + r1 * 32 + lane;
-#pragma unroll 2
+        // partial rows are stored with chunk c of row m at position c ^ (m & 7)
+        const float4 *v = gbuf + r * 32 + (lane ^ ((r_lo + r) & 7));
+        const float4 *u = gbuf + r1 * 32 + (lane ^ ((r_lo + r1) & 7));
+#pragma unroll 4
         for (int q = 0; q < sp.n; ++q, v += nr * 32, u += nr * 32) {
             const float2 w = make_float2(wsm[q], wsm[q]), z = make_float2(wsm[sp.n + q], wsm[sp.n + q]);
             const float4 x = *v, y = *u;
@@ -833,7 +1085,7 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
 }
 
 __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem, const AttnArgs &p,
-                                                 const Decomp &d, int cid, uint32_t tmem)
+                                                 const Plan &pl, int cid, uint32_t tmem)
 {
     const int warp = threadIdx.x >> 5;          // 0..3 = TMEM lane quarter
     const int lane = threadIdx.x & 31;
@@ -846,12 +1098,8 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.scale_log2;
 
-    PieceIter it(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, d, cid);
-    if (threadIdx.x == 0) {                      // for the split merge
-        reinterpret_cast<int64_t *>(smem + kSmemPend)[0] = d.W;
-        reinterpret_cast<int *>(smem + kSmemPend)[2] = d.P;
-    }
-    Piece pc;
+    BoxIter it(pl, p);
+    TPiece pc;
     uint32_t gt = 0, qp = 0, piece = 0, epi = 0;
     int npend = 0;                               // shared segments awaiting the merge
     uint32_t gph = 0;                            // B_GATHER phases used
@@ -862,7 +1110,7 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
         ++epi;
         return ok;
     };
-    while (it.next(pc)) {
+    while (next_piece(it, pc)) {
         const int C = pc.len - p.K;
         const int lim = p.view == ORTHRUS_AR ? C + i : 0x7FFFFFFF;   // last visible key
         const Tiling tl(pc.a, pc.e);
@@ -963,6 +1211,7 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
             tc_fence_after();
         }
         const bool sole = pc.a == 0 && pc.e == pc.len;
+        const bool last = pc.s0 + nbox_of(pc.e) == pl.hi;     // the range's last piece
         const size_t slot = (size_t)cid + pc.s;
         if (!sole && npend < 2) {
             // (only the first and the last piece of a range can be shared;
@@ -970,11 +1219,12 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
             if (threadIdx.x == 0) {
                 SharedPiece sp;
                 sp.s0 = pc.s0;
+                sp.nbx = pc.nbx;
                 sp.b = pc.b;
                 sp.g = pc.g;
                 sp.s = pc.s;
-                sp.len = pc.len;
-                reinterpret_cast<SharedPiece *>(smem + kSmemPend + 16)[npend] = sp;
+                sp.idx = (int)piece;
+                reinterpret_cast<SharedPiece *>(smem + kSmemPend)[npend] = sp;
             }
             ++npend;
         }
@@ -983,60 +1233,84 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
             // zero output, zero weight in the merge
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             const float2 inv2 = make_float2(inv, inv);
-            float4 *srow = reinterpret_cast<float4 *>(smem + kSmemStage) + m * (kStagePitch / 4);
+            // the O row in four chunks of 32 columns (TMEM load, wait, scale, stage)
+            auto stage_row = [&](float4 *srow, int swz) {
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + kColO + 32 * ch, o);
-                tmem_wait_ld();
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + kColO + 32 * ch, o);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float2 x = fmul2(make_float2(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1])), inv2);
-                    const float2 y = fmul2(make_float2(__uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3])), inv2);
-                    srow[8 * ch + c] = make_float4(x.x, x.y, y.x, y.y);
+                    for (int c = 0; c < 8; ++c) {
+                        const float2 x = fmul2(make_float2(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1])), inv2);
+                        const float2 y = fmul2(make_float2(__uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3])), inv2);
+                        srow[(8 * ch + c) ^ swz] = make_float4(x.x, x.y, y.x, y.y);
+                    }
                 }
-            }
-            fence_proxy_async();                  // the row is visible to the bulk copy
-            if (row_ok) {
-                float *dst = sole ? p.out + (((size_t)pc.b * p.K + i) * p.Hq + pc.g * G + m % G) * kD
-                                  : p.ws_o + (slot * rows + m) * kD;
-                bulk_store(dst, sh.base + kSmemStage + m * kStagePitch * 4, kD * 4);
-                bulk_commit();
-                if (!sole) p.ws_lse[slot * lse_pitch(rows) + m] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+            };
+            if (sole) {
+                // final rows: padded staging (conflict-free), one bulk copy per row
+                stage_row(reinterpret_cast<float4 *>(smem + kSmemStage) + m * (kStagePitch / 4), 0);
+                fence_proxy_async();              // the row is visible to the bulk copy
+                if (row_ok) {
+                    bulk_store(p.out + (((size_t)pc.b * p.K + i) * p.Hq + pc.g * G + m % G) * kD,
+                               sh.base + kSmemStage + m * kStagePitch * 4, kD * 4);
+                    bulk_commit();
+                }
+            } else {
+                // a partial: rows contiguous in the workspace, staged unpadded
+                // with chunk c of row m at position c ^ (m & 7) (conflict-free),
+                // one bulk copy per warp; the merge reads the same swizzle
+                stage_row(reinterpret_cast<float4 *>(smem + kSmemStage) + m * 32, m & 7);
+                fence_proxy_async();              // the rows are visible to the bulk copy
+                __syncwarp();
+                if (lane == 0) {
+                    const int r0 = warp * 32, nrow = rows - r0 < 32 ? rows - r0 : 32;
+                    bulk_store(p.ws_o + (slot * rows + r0) * kD, sh.base + kSmemStage + r0 * kD * 4,
+                               (uint32_t)nrow * kD * 4);
+                    bulk_commit();
+                }
+                if (row_ok) p.ws_lse[slot * lse_pitch(rows) + m] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
             }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sh.bar(B_OFREE));          // TMEM O may be overwritten
         ++qp;
+        if (!sole && warp_ok && lane == 0) {
+            // publish this warp's rows of the partial: written (with the warp's
+            // log2-sum-exp values, ordered by the __syncwarp above), then its
+            // flag += 1 (release); the partial is complete at ceil(rows / 32)
+            bulk_wait_all();
+            fence_proxy_async_global();
+            counter_add_release(p.ws_sync + (last ? kSyncLast : kSyncFirst) * kMaxSyncUnits + cid, 1);
+        }
+        ++piece;
+        if (last) break;                                      // (no next piece: nothing refills the rings)
         bulk_wait_read();                                     // the staging row has been read
         if (!epi_sync()) return false;
         if (threadIdx.x == 0) mbar_arrive(sh.bar(B_MERGED)); // the rings may be refilled
-        ++piece;
     }
     bulk_wait_all();                                          // rows written
     if (npend == 0) return true;
 
-    // ---- split merge: every CTA of a shared segment publishes its partial
-    // (arrive[c_lo] += 1, release), then merges its share of the segment's
-    // rows (split_merge)
-    fence_proxy_async_global();                               // bulk writes before
-    if (!epi_sync()) return false;                            // the release below
-    Decomp ds;                                                // (the split, from shared memory)
-    ds.W = reinterpret_cast<const int64_t *>(smem + kSmemPend)[0];
-    ds.P = reinterpret_cast<const int *>(smem + kSmemPend)[2];
+    // ---- split merge: this CTA's share of the rows of each shared segment
+    // (split_merge); the gathers overwrite the staging area, which every
+    // warp's copies have read by now (bulk_wait_all above, then this join)
+    if (!epi_sync()) return false;
+    const Plan plan = *reinterpret_cast<const Plan *>(smem + kSmemPlan);
     auto shared_piece = [&](int k) {
-        const SharedPiece sp = reinterpret_cast<const SharedPiece *>(smem + kSmemPend + 16)[k];
+        const SharedPiece sp = reinterpret_cast<const SharedPiece *>(smem + kSmemPend)[k];
         SplitInfo si;
         si.b = sp.b;
         si.g = sp.g;
         si.s = sp.s;
-        si.c_lo = cta_of(ds, sp.s0);
-        si.n = cta_of(ds, sp.s0 + sp.len - 1) - si.c_lo + 1;
+        si.c_lo = plan_cta_of(plan, sp.s0);
+        const int c_hi = plan_cta_of(plan, sp.s0 + sp.nbx - 1);
+        si.n = c_hi - si.c_lo + 1;
+        si.hi_last = plan_start(plan, c_hi + 1) <= sp.s0 + sp.nbx;
         return si;
     };
-    if (threadIdx.x == 0)
-        for (int k = 0; k < npend; ++k) counter_add_release(p.ws_sync + shared_piece(k).c_lo, 1);
     for (int k = 0; k < npend; ++k) {
         if (k > 0 && !epi_sync()) return false;               // gather buffer free again
         const SplitInfo sp = shared_piece(k);
@@ -1109,23 +1383,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- everything below may read what earlier kernels wrote
     pdl_wait();
-    const Decomp d = make_decomp(p.ctx_lens, p.B, p.Hkv, p.K, p.S_max, gridDim.x, p.min_keys);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        for (int b = 0; b < p.B; ++b)
-            if (seg_len(p.ctx_lens, b, p.K, p.S_max) == 0) raise_status(p.status, ORTHRUS_STATUS_CAPACITY);
+    Plan *plan_s = reinterpret_cast<Plan *>(base_ptr + kSmemPlan);
+    if (warp == 4) {
+        const PlanArgs pa = {p.ctx_lens, p.status, p.B, p.Hkv, p.K, p.S_max};
+        plan_prologue(pa, p.ws_plan, gridDim.x, cid, p.min_keys > kBoxKeys ? p.min_keys / kBoxKeys : 1, plan_s);
     }
-    if (d.W > 0 && cid < d.P) {
+    __syncthreads();
+    const Plan pl = *plan_s;
+    if (pl.NB > 0 && cid < pl.P) {
         if (warp < 4) {
-            softmax_epilogue(sh, base_ptr, p, d, cid, tmem);
+            softmax_epilogue(sh, base_ptr, p, pl, cid, tmem);
             bulk_wait_all();                      // (also after an abort)
         } else if (warp == 4) {
-            if (lane == 0) producer(sh, p, d, cid, &tm_q, &tm_k, &tm_v);
+            if (lane == 0) producer(sh, p, pl, &tm_q, &tm_k, &tm_v);
             __syncwarp();
         } else if (warp == 5) {
-            if (lane == 0) s_issuer(sh, p, d, cid, tmem);
+            if (lane == 0) s_issuer(sh, p, pl, tmem);
             __syncwarp();
         } else {
-            if (lane == 0) pv_issuer(sh, p, d, cid, tmem);
+            if (lane == 0) pv_issuer(sh, p, pl, tmem);
             __syncwarp();
         }
     }

@@ -15,7 +15,8 @@ struct AttnArgs {
     const void *v_cache;
     const int32_t *ctx_lens;
     float *out;
-    int32_t *ws_sync;    // [2, kMaxSyncUnits] split-merge counters (zero between calls)
+    int32_t *ws_sync;    // [3, kMaxSyncUnits] split-merge flags and counters (zero between calls)
+    int32_t *ws_plan;    // [kMaxSyncUnits, kPlanEntryInts] per-CTA cached work plans
     float *ws_o;         // [slots, rows, D] split partials (O normalised)
     float *ws_lse;       // [slots, lse_pitch(rows)] log2-sum-exp of each partial
     int32_t *status;
@@ -26,13 +27,24 @@ struct AttnArgs {
     int min_keys;        // smallest key range worth a CTA
 };
 
-// Workspace layout shared by the attention paths: a fixed block of counters
-// used by the tensor-core path's in-kernel split merge (arrive[u], depart[u]
-// for the split unit u that opens a segment; zero before and after every
-// call), then `slots` fp32 partial tiles [rows, D], then their log2-sum-exp
-// values [rows].
+// Workspace layout shared by the attention paths: a fixed block of flags and
+// counters used by the tensor-core path's in-kernel split merge (zero before
+// and after every call):
+//   first[u]  unit u has published the partial of the first piece of its range
+//             (set only when that piece is shared and is not also its last)
+//   last[u]   unit u has published the partial of the last piece of its range
+//   depart[u] units done reading the flags of the segment that unit u opens
+// then `slots` fp32 partial tiles [rows, D], then their log2-sum-exp values.
 constexpr int kMaxSyncUnits = 160;     // >= the tensor-core path's CTA count (148 on B200)
-constexpr size_t kSyncBytes = 2 * kMaxSyncUnits * sizeof(int32_t);
+constexpr int kSyncFirst = 0, kSyncLast = 1, kSyncDepart = 2;
+constexpr size_t kSyncBytes = 3 * kMaxSyncUnits * sizeof(int32_t);
+// After it, one cached work plan per CTA of the tensor-core path: the split
+// of the key space that CTA computed, keyed by the shape and the context
+// lengths it was computed for (batches of up to kPlanMaxB sequences), so that
+// a later call with the same lengths loads it instead of recomputing it.
+constexpr int kPlanMaxB = 32;
+constexpr int kPlanEntryInts = 64;     // key (8) + lengths (32) + plan (10), padded
+constexpr size_t kPlanBytes = (size_t)kMaxSyncUnits * kPlanEntryInts * sizeof(int32_t);
 inline size_t attn_ws_o_bytes(int slots, int rows, int D)
 {
     return ((size_t)slots * rows * D * sizeof(float) + 255) & ~(size_t)255;
@@ -45,7 +57,7 @@ inline size_t attn_ws_lse_bytes(int slots, int rows)
 }
 inline size_t attn_ws_bytes(int slots, int rows, int D)
 {
-    return kSyncBytes + attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
+    return kSyncBytes + kPlanBytes + attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
 }
 
 cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);

@@ -20,6 +20,9 @@ from gpu_util import assert_attn_close, run_attn, tdtype, to_dev
 
 pytestmark = pytest.mark.gpu
 
+# the workspace's leading block of split-merge flags and counters: 3 x 160 int32
+SYNC_BYTES = 3 * 160 * 4
+
 
 @functools.lru_cache(maxsize=2)
 def _inputs(name, layer, view):
@@ -168,7 +171,8 @@ def test_repeatable_bitwise():
 def test_workspace_reused_across_calls_and_shapes():
     """One workspace, zero-filled once, serves consecutive calls of different
     context lengths, views and batch shapes: every call matches the oracle and
-    leaves the split-merge counter block (the workspace's first 1280 bytes)
+    leaves the split-merge flag and counter block (the workspace's first 1920
+    bytes)
     zero again."""
     cases = [(11, 1, [5000]), (12, 2, [3000, 700]), (13, 3, [1, 2500, 129]), (14, 1, [200])]
     need = max(ob.orthrus_attn_workspace_size(B, 32, 8, 128, 32, torch.bfloat16) for _, B, _ in cases)
@@ -183,15 +187,15 @@ def test_workspace_reused_across_calls_and_shapes():
                             status=status)
             torch.cuda.synchronize()
             assert int(status.item()) == 0
-            assert int(ws[:1280].count_nonzero().item()) == 0, "split-merge counters left set"
+            assert int(ws[:SYNC_BYTES].count_nonzero().item()) == 0, "split-merge flags left set"
             assert_attn_close(out.cpu().numpy(), oracle.attention(view, q, kc, vc, ctx),
                               f"reuse B={B} view={view}")
 
 
 def test_merge_wait_gives_up_on_counters_that_never_complete():
-    """A workspace whose split-merge counters were not zeroed (documented
-    misuse): every split segment's merge waits for a count that can never
-    arrive, gives up after its bound, and the call sets ORTHRUS_STATUS_TIMEOUT
+    """A workspace whose split-merge flags were not zeroed (documented misuse):
+    every split segment's merge waits for a publish flag that can never reach
+    one, gives up after its bound, and the call sets ORTHRUS_STATUS_TIMEOUT
     instead of hanging or faulting; the context stays usable and the next call
     on a zeroed workspace is exact."""
     q, kc, vc, ctx = _custom(15, 1, 32, 8, 128, 32, [5000])     # every segment split
@@ -199,7 +203,7 @@ def test_merge_wait_gives_up_on_counters_that_never_complete():
     c = torch.from_numpy(ctx).cuda()
     need = ob.orthrus_attn_workspace_size(1, 32, 8, 128, 32, torch.bfloat16)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    ws[:640].view(torch.int32).fill_(-1_000_000)                # arrive counters
+    ws[:2 * SYNC_BYTES // 3].view(torch.int32).fill_(-1_000_000)   # publish flags
     out = torch.empty((1, 32, 32, 128), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ob.orthrus_attn(ob.DIFF, *args, c, out, ws, status=status)
