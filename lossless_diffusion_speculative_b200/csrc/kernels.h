@@ -1,6 +1,7 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -59,6 +60,11 @@ inline size_t attn_ws_bytes(int slots, int rows, int D)
 {
     return kSyncBytes + kPlanBytes + attn_ws_o_bytes(slots, rows, D) + attn_ws_lse_bytes(slots, rows);
 }
+
+// TMA tensor map of a bf16 tensor with 128-byte swizzle: dims[0] innermost
+// (elements), strides[i] = bytes between consecutive indices of dimension i+1.
+bool encode_bf16_sw128(CUtensorMap *m, int rank, const void *base, const uint64_t *dims,
+                       const uint64_t *strides, const uint32_t *box);
 
 cudaError_t launch_attn_simt(const AttnArgs &p, int grid, cudaStream_t st);
 cudaError_t launch_attn_combine(const AttnArgs &p, int grid_main, cudaStream_t st);

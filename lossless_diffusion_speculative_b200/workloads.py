@@ -29,6 +29,7 @@ T_Q = {0: 3, 1: 6}          # view -> query tensor id (0 = DIFF, 1 = AR)
 T_K_BLK = {0: 4, 1: 7}
 T_V_BLK = {0: 5, 1: 8}
 T_LOGITS, T_PLANT = 9, 10   # consensus inputs (layer index 99)
+T_HIDDEN, T_LMHEAD, T_LMPLANT = 11, 12, 13   # fused LM-head inputs (layer index 97)
 
 
 @dataclass(frozen=True)
@@ -51,6 +52,7 @@ class Workload:
     value_scale: float         # Q/K/V ~ N(0,1) * value_scale
     extra_rows: int = -1       # cache rows beyond max(ctx)+K (default: K)
     note: str = ""
+    hidden: int = 4096         # model width (the AR LM head's input size)
 
     @property
     def G(self) -> int:
@@ -89,12 +91,12 @@ _INV_SQRT_128 = 1.0 / np.sqrt(128.0)
 WORKLOADS = {
     "tiny_f32": Workload(1, "tiny_f32", B=1, Hq=4, Hkv=2, D=64, K=8, layers=1,
                          dtype="f32", vocab=1000, logit_sigma=1.0, plant="fixed:3",
-                         ctx_lo=256, ctx_hi=256, value_scale=1.0,
+                         ctx_lo=256, ctx_hi=256, value_scale=1.0, hidden=256,
                          note="tiny single step, fp32, 1 layer"),
     "qwen3_1p7b_layer": Workload(2, "qwen3_1p7b_layer", B=1, Hq=16, Hkv=8, D=128, K=32,
                                  layers=1, dtype="bf16", vocab=151936, logit_sigma=2.0,
                                  plant="geom:0.14285714285714285", ctx_lo=4096,
-                                 ctx_hi=4096, value_scale=_INV_SQRT_128,
+                                 ctx_hi=4096, value_scale=_INV_SQRT_128, hidden=2048,
                                  note="Qwen3-1.7B-shaped single layer"),
     "qwen3_8b_step": Workload(3, "qwen3_8b_step", B=1, Hq=32, Hkv=8, D=128, K=32,
                               layers=36, dtype="bf16", vocab=151936, logit_sigma=2.0,
@@ -104,7 +106,7 @@ WORKLOADS = {
     "qwen3_4b_ragged": Workload(4, "qwen3_4b_ragged", B=16, Hq=32, Hkv=8, D=128, K=32,
                                 layers=1, dtype="bf16", vocab=151936, logit_sigma=2.0,
                                 plant="geom:0.1111111111111111", ctx_lo=2048,
-                                ctx_hi=16384, value_scale=_INV_SQRT_128,
+                                ctx_hi=16384, value_scale=_INV_SQRT_128, hidden=2560,
                                 note="Qwen3-4B-shaped ragged batch of 16"),
     "qwen3_8b_long_k8": Workload(5, "qwen3_8b_long_k8", B=4, Hq=32, Hkv=8, D=128, K=8,
                                  layers=1, dtype="bf16", vocab=151936, logit_sigma=2.0,
@@ -275,3 +277,50 @@ def consensus_inputs(w: Workload, accept: Optional[np.ndarray] = None,
             prop[b, a[b]] = (r[b, a[b]] + 1 + rng.integers(0, V - 1)) % V
     nxt = r[np.arange(B), np.minimum(a, K - 1)].astype(np.int32)
     return ConsensusInputs(logits, prop, r, a.astype(np.int32), nxt)
+
+
+@dataclass
+class LMHeadInputs:
+    hidden: np.ndarray          # [B, K, Hd] float32 holding bf16 values
+    lm_head: np.ndarray         # [V, Hd] float32 holding bf16 values
+    proposed: np.ndarray        # [B, K] int32
+    planted_argmax: np.ndarray  # [B, K] int32
+    planted_accept: np.ndarray  # [B] int32
+    planted_next: np.ndarray    # [B] int32
+
+
+def lm_head_inputs(w: Workload, Hd: Optional[int] = None, V: Optional[int] = None,
+                   accept: Optional[np.ndarray] = None, plant: bool = True) -> LMHeadInputs:
+    """Inputs of the fused AR LM head + consensus: the AR view's final hidden
+    states h [B, K, Hd] ~ N(0, 1) and a weight W [V, Hd] ~ N(0, 1/Hd), both
+    rounded to bf16 (random logits ~ N(0, 1)).
+
+    With ``plant``, every token row t gets its own planted token r_t (distinct)
+    whose weight row is W[r_t] = 12 h_t / |h_t|^2: its logit is 12, far above
+    the random ones (max ~ 4.6 over 151936) and the other planted rows' cross
+    terms (~ 12 / sqrt(Hd) std), so the argmax is known; the proposals match it
+    on exactly the first a_b slots (the workload's acceptance law)."""
+    Hd = w.hidden if Hd is None else Hd
+    V = w.vocab if V is None else V
+    B, K = w.B, w.K
+    rng = _rng(w, 97, T_HIDDEN)
+    h = round_to_bf16(rng.standard_normal((B, K, Hd), dtype=np.float32))
+    W = _rng(w, 97, T_LMHEAD).standard_normal((V, Hd), dtype=np.float32)
+    W *= np.float32(1.0 / np.sqrt(Hd))
+    W = round_to_bf16(W)
+    prng = _rng(w, 97, T_LMPLANT)
+    r = prng.choice(V, size=B * K, replace=False).astype(np.int32) if plant else \
+        np.zeros(B * K, np.int32)
+    if plant:
+        hf = h.reshape(B * K, Hd).astype(np.float64)
+        rows = 12.0 * hf / (hf * hf).sum(axis=1, keepdims=True)
+        W[r] = round_to_bf16(rows.astype(np.float32))
+    r = r.reshape(B, K)
+    a = planted_accept_lengths(w) if accept is None else np.asarray(accept, np.int32)
+    prop = prng.integers(0, V, size=(B, K)).astype(np.int32)
+    for b in range(B):
+        prop[b, :a[b]] = r[b, :a[b]]
+        if a[b] < K:
+            prop[b, a[b]] = (r[b, a[b]] + 1 + prng.integers(0, V - 1)) % V
+    nxt = r[np.arange(B), np.minimum(a, K - 1)].astype(np.int32)
+    return LMHeadInputs(h, W, prop, r, a.astype(np.int32), nxt)

@@ -4,9 +4,11 @@ TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
 and by the CPU-baseline leg of ``bench.py``.  The product library never imports,
 links or calls it, and it shares no code with the CUDA path.
 
-The arithmetic lives in ``orthrus_oracle.c`` (plain C, double precision,
-OpenMP over output rows).  This module only compiles it with gcc and marshals
-numpy arrays through ctypes.  Each function follows the technical summary of
+The attention, consensus and commit arithmetic lives in ``orthrus_oracle.c``
+(plain C, double precision, OpenMP over output rows); this module compiles it
+with gcc and marshals numpy arrays through ctypes.  The fused LM-head consensus
+(``lm_head_consensus``) is numpy in float64: one library matrix product for the
+logits, then the argmax and the prefix walk written out here.  Each function follows the technical summary of
 "Orthrus: Memory-Efficient Parallel Token Generation via Dual-View Diffusion"
 (gist.science page), sections 2.2 (mask M_diff) and 2.3 (verification,
 consensus and commitment); see the C file's header for the readings taken
@@ -154,3 +156,61 @@ def kv_commit(k_cache: np.ndarray, v_cache: np.ndarray, k_blk, v_blk,
         B, Hkv, D, S_max, K, k_cache.dtype.itemsize, 1 if advance else 0)
     if rc != 0:
         raise ValueError("oracle_kv_commit: bad argument or capacity violation")
+
+
+def lm_head_logits(hidden: np.ndarray, lm_head: np.ndarray) -> np.ndarray:
+    """float64 logits[t, v] = <hidden[t], lm_head[v]> for token rows t = b*K + i.
+
+    The AR head scores every block position in one pass ("Orthrus: Memory-
+    Efficient Parallel Token Generation via Dual-View Diffusion", gist.science
+    technical summary, section 2.3 "structural verification").  hidden
+    [B, K, Hd] and lm_head [V, Hd] hold bf16 values exactly (float32 arrays);
+    the product is taken in float64 (a library matmul), so every logit is
+    within ~1e-16 relative of the exact dot product.
+    """
+    B, K, Hd = hidden.shape
+    V, Hd2 = lm_head.shape
+    assert Hd2 == Hd
+    h = np.asarray(hidden, np.float64).reshape(B * K, Hd)
+    return h @ np.asarray(lm_head, np.float64).T
+
+
+def lm_head_consensus(hidden: np.ndarray, lm_head: np.ndarray, proposed: np.ndarray):
+    """Greedy consensus on the AR head's logits, never materialised on the GPU.
+
+    r[b, i] = argmax_v logits[b*K + i, v] (lowest index wins ties), then the
+    left-to-right prefix walk of section 2.3 "consensus and commitment": a =
+    number of leading i with proposed[b, i] == r[b, i]; next = r[b, min(a, K-1)].
+
+    Returns (accepted [B], next [B], argmax [B, K], gap [B, K], absdot [B, K])
+    where gap is the float64 difference between each row's largest and second
+    largest logit and absdot = max_v sum_d |hidden[t, d] * lm_head[v, d]|, the
+    scale of the rounding error of a float32 accumulation of that row.
+    """
+    B, K, Hd = hidden.shape
+    logits = lm_head_logits(hidden, lm_head)
+    r = np.argmax(logits, axis=1)                       # first maximum = lowest index
+    top2 = np.partition(logits, logits.shape[1] - 2, axis=1)[:, -2:] if logits.shape[1] > 1 else None
+    gap = (top2[:, 1] - top2[:, 0]) if top2 is not None else np.full(B * K, np.inf)
+    absdot = (np.abs(np.asarray(hidden, np.float64).reshape(B * K, Hd))
+              @ np.abs(np.asarray(lm_head, np.float64)).T).max(axis=1)
+    r = r.reshape(B, K).astype(np.int32)
+    acc = np.empty(B, np.int32)
+    nxt = np.empty(B, np.int32)
+    for b in range(B):
+        a = 0
+        while a < K and int(proposed[b, a]) == int(r[b, a]):
+            a += 1
+        acc[b] = a
+        nxt[b] = r[b, min(a, K - 1)]
+    return acc, nxt, r, gap.reshape(B, K), absdot.reshape(B, K)
+
+
+def fp32_dot_error_bound(n: int, absdot) -> np.ndarray:
+    """Rigorous bound on |fl32(sum) - sum| for a float32 accumulation of n
+    exact products (bf16 x bf16 products are exact in float32) in any order,
+    with rounding to nearest or toward zero: gamma_n * sum |x_d y_d|, gamma_n =
+    n*u / (1 - n*u), u = 2^-23 (the toward-zero unit, twice round-to-nearest's).
+    """
+    u = 2.0 ** -23
+    return n * u / (1.0 - n * u) * np.asarray(absdot, np.float64)

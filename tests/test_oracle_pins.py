@@ -371,3 +371,87 @@ def test_lossless_toy_loop_equals_greedy(mode):
             assert a == K
     out = (seq + [anchor])[:len(prompt) + steps_tokens]
     assert out == greedy[:len(out)]
+
+
+# --------------------------------------------------------------------------- fused LM head
+
+def _lm_case(seed, B=2, K=4, Hd=32, V=50):
+    rng = np.random.default_rng(seed)
+    h = wl.round_to_bf16(rng.standard_normal((B, K, Hd), dtype=np.float32))
+    W = wl.round_to_bf16(rng.standard_normal((V, Hd), dtype=np.float32) / np.float32(np.sqrt(Hd)))
+    return h, W
+
+
+def test_lm_head_bruteforce_tiny():
+    """Explicit loops: dot products, first maximum, left-to-right prefix walk."""
+    h, W = _lm_case(40)
+    B, K, Hd = h.shape
+    V = W.shape[0]
+    rng = np.random.default_rng(41)
+    prop = rng.integers(0, V, (B, K)).astype(np.int32)
+    r_bf = np.zeros((B, K), np.int32)
+    for b in range(B):
+        for i in range(K):
+            best, arg = -math.inf, -1
+            for v in range(V):
+                dot = math.fsum(float(h[b, i, d]) * float(W[v, d]) for d in range(Hd))
+                if dot > best:
+                    best, arg = dot, v
+            r_bf[b, i] = arg
+    prop[0, :2] = r_bf[0, :2]                     # sequence 0 accepts 2, sequence 1 all K
+    prop[0, 2] = (r_bf[0, 2] + 1) % V
+    prop[1, :] = r_bf[1, :]
+    acc, nxt, r, _, _ = oracle.lm_head_consensus(h, W, prop)
+    assert (r == r_bf).all()
+    assert acc[0] == 2 and nxt[0] == r_bf[0, 2]
+    assert acc[1] == K and nxt[1] == r_bf[1, K - 1]
+
+
+@pytest.mark.parametrize("a", [0, 5, 32])
+def test_lm_head_recovers_plant(a):
+    w = wl.WORKLOADS["qwen3_8b_step"].with_(vocab=3000)
+    li = wl.lm_head_inputs(w, Hd=128, accept=np.array([a], np.int32))
+    acc, nxt, r, gap, _ = oracle.lm_head_consensus(li.hidden, li.lm_head, li.proposed)
+    assert (r == li.planted_argmax).all()
+    assert acc[0] == a and nxt[0] == li.planted_next[0]
+    assert gap.min() > 1.0
+
+
+def test_lm_head_matches_materialised_consensus():
+    """The fused definition and the C consensus over materialised (float32)
+    logits agree wherever the top-2 gap dwarfs float32 rounding."""
+    w = wl.WORKLOADS["qwen3_4b_ragged"].with_(B=3, vocab=2000)
+    li = wl.lm_head_inputs(w, Hd=96)
+    acc, nxt, r, gap, _ = oracle.lm_head_consensus(li.hidden, li.lm_head, li.proposed)
+    logits = oracle.lm_head_logits(li.hidden, li.lm_head).astype(np.float32).reshape(3, w.K, -1)
+    acc2, nxt2, r2 = oracle.consensus(logits, li.proposed)
+    assert gap.min() > 1e-3
+    assert (acc == acc2).all() and (nxt == nxt2).all() and (r == r2).all()
+
+
+def test_lm_head_ties_go_to_the_lowest_index():
+    h, W = _lm_case(42, B=1, K=2, Hd=16, V=20)
+    W[7] = W[3] = h[0, 0] * 4                     # two equal maxima for row 0
+    prop = np.array([[3, 0]], np.int32)
+    acc, nxt, r, gap, _ = oracle.lm_head_consensus(h, W, prop)
+    assert r[0, 0] == 3 and gap[0, 0] == 0.0 and acc[0] >= 1
+
+
+def test_fp32_accumulation_stays_within_the_stated_bound():
+    """float32 sums of the exact products in several orders never leave the
+    bound the GPU parity tests use to decide which argmaxes are unique."""
+    rng = np.random.default_rng(43)
+    for n in (64, 1000, 4096):
+        x = wl.round_to_bf16(rng.standard_normal(n, dtype=np.float32))
+        y = wl.round_to_bf16(rng.standard_normal(n, dtype=np.float32) * np.float32(3))
+        prod = (x.astype(np.float64) * y.astype(np.float64))
+        exact = math.fsum(prod)
+        bound = float(oracle.fp32_dot_error_bound(n, np.abs(prod).sum()))
+        p32 = prod.astype(np.float32)                 # exact: bf16 x bf16 fits in float32
+        assert (p32.astype(np.float64) == prod).all()
+        for order in (p32, p32[::-1], np.sort(p32), rng.permutation(p32)):
+            acc = np.float32(0)
+            for v in order:
+                acc = np.float32(acc + v)
+            assert abs(float(acc) - exact) <= bound
+        assert abs(float(np.sum(p32, dtype=np.float32)) - exact) <= bound
