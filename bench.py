@@ -311,6 +311,70 @@ def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
     return out
 
 
+# ----------------------------------------------------------------------------- fused LM head
+LM_HEAD_SET = ("qwen3_1p7b_layer", "qwen3_8b_step", "qwen3_4b_ragged", "qwen3_8b_long_k32")
+
+
+def measure_lm_head(name, dev, stream, hbm, iters):
+    """orthrus_lm_head_consensus on the workload's Qwen3 width and vocabulary:
+    median µs per call over `iters` calls with L2 flushed before each, and the
+    weight-read bandwidth (the [V, Hd] bf16 weight is the algorithmic traffic;
+    hidden states, proposals and outputs are < 0.5 %).  Inputs are drawn on the
+    device from a seeded torch generator (random N(0, 1/Hd) weights, N(0, 1)
+    hidden states, one planted argmax per token row, proposals matching the
+    plant on the workload's planted acceptance length)."""
+    import torch
+    from lossless_diffusion_speculative_b200 import binding as ob
+    from lossless_diffusion_speculative_b200 import workloads as wl
+
+    w = wl.WORKLOADS[name]
+    B, K, V, Hd = w.B, w.K, w.vocab, w.hidden
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 * w.cid + 97)
+    W = (torch.randn((V, Hd), generator=g, device=dev) * (1.0 / Hd ** 0.5)).to(torch.bfloat16)
+    h = torch.randn((B * K, Hd), generator=g, device=dev).to(torch.bfloat16)
+    r = torch.randperm(V, generator=g, device=dev)[:B * K]
+    hf = h.float()
+    W[r] = (12.0 * hf / (hf * hf).sum(dim=1, keepdim=True)).to(torch.bfloat16)
+    a = torch.from_numpy(wl.planted_accept_lengths(w)).to(dev)
+    prop = torch.randint(0, V, (B, K), generator=g, device=dev, dtype=torch.int32)
+    rr = r.view(B, K).to(torch.int32)
+    slot = torch.arange(K, device=dev)[None, :]
+    prop = torch.where(slot < a[:, None], rr, prop)
+    prop = torch.where(slot == a[:, None], (rr + 1) % V, prop).contiguous()
+    h = h.view(B, K, Hd).contiguous()
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    nxt = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = torch.zeros(ob.orthrus_lm_head_workspace_size(B, K), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for it in range(3 + iters):
+            flush.zero_()
+            if it >= 3:
+                ev[it - 3][0].record()
+            ob.orthrus_lm_head_consensus(h, W, prop, acc, nxt, ws, status=status, stream=stream)
+            if it >= 3:
+                ev[it - 3][1].record()
+        torch.cuda.synchronize()
+    exp_a = torch.clamp(a, max=K).to(torch.int32)
+    if int(status.item()) != 0 or not torch.equal(acc, exp_a):
+        raise RuntimeError(f"lm_head {name}: status {int(status.item()):#x}, accepted {acc.tolist()}")
+    us = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev])) * 1e3
+    wbytes = V * Hd * 2
+    gbs = wbytes / (us * 1e-6) / 1e9
+    flops = 2.0 * B * K * Hd * V
+    out = {"workload": name, "B": B, "K": K, "V": V, "Hd": Hd, "us_per_call": us,
+           "weight_bytes": wbytes, "weight_read_gbs": gbs, "frac_of_hbm": gbs / hbm,
+           "tflops": flops / (us * 1e-6) / 1e12, "iters": iters,
+           "kernel": "lm_head_kernel (tcgen05 swap-AB GEMM, argmax epilogue, last-CTA consensus)",
+           "timing": "median of CUDA events per call; L2 flushed before each call"}
+    del W, h, flush
+    return out
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse()
@@ -482,6 +546,10 @@ def main():
                 configs[label] = measure_config(label, wl.WORKLOADS[name], order, dev, stream,
                                                 hbm, CONFIG_ITERS,
                                                 st=st if name == w.name else None)
+                torch.cuda.empty_cache()
+            for name in LM_HEAD_SET:
+                configs["lm_head_consensus_" + name] = measure_lm_head(name, dev, stream, hbm,
+                                                                       CONFIG_ITERS)
                 torch.cuda.empty_cache()
         torch.cuda.synchronize()
         clocks = sampler.stop()

@@ -270,6 +270,55 @@ ORTHRUS_API int orthrus_attn_static(orthrus_view view, orthrus_dtype dtype, cons
                                     int S_max, int K, float scale, float *out, int32_t *status,
                                     void *stream);
 
+/*
+ * orthrus_lm_head_workspace_size — bytes of scratch orthrus_lm_head_consensus
+ * needs: one 8-byte running maximum per token row plus a completion counter.
+ * Returns 0 for invalid sizes (B * K above ORTHRUS_MAX_LM_ROWS).
+ */
+#define ORTHRUS_MAX_LM_ROWS 512
+ORTHRUS_API size_t orthrus_lm_head_workspace_size(int B, int K);
+
+/*
+ * orthrus_lm_head_consensus — the AR view's LM head fused with the greedy
+ * consensus (section 2.3 "structural verification": the frozen AR head scores
+ * all K block positions in one pass; "consensus and commitment": strict
+ * left-to-right acceptance, the AR token replaces the first mismatch).  The
+ * [B, K, V] logits are never written to memory.
+ *
+ * For token row t = b * K + i:
+ *     logits[t, v] = sum_d hidden[b, i, d] * lm_head[v, d]   (fp32 accumulation)
+ *     r[b, i]      = argmax_v logits[t, v]   (lowest index wins ties; NaN ranks
+ *                    above every number, the first NaN wins; +0 == -0)
+ * then, exactly as orthrus_consensus: accepted_len[b] = number of leading i
+ * with proposed[b, i] == r[b, i], in [0, K]; next_token[b] = r[b, min(a, K-1)].
+ *
+ *   hidden       [B, K, Hd] bf16: the AR view's final hidden states (after the
+ *                model's final norm); row i scores the token after block slot i.
+ *   lm_head      [V, Hd] bf16: the output projection, one row per vocabulary
+ *                entry (Hd contiguous).
+ *   proposed     [B, K] int32 diffusion-view proposals.
+ *   accepted_len [B] int32 out; next_token [B] int32 out; argmax_out optional
+ *                [B, K] int32 out (r itself, may be NULL).
+ *   workspace    >= orthrus_lm_head_workspace_size(B, K) bytes, 16-byte
+ *                aligned.  Zero-fill it once before its first use: the call
+ *                needs it zero when it starts and leaves it zero when it
+ *                completes.  A call that ended with ORTHRUS_STATUS_TIMEOUT may
+ *                leave it set: zero it again.  Calls that overlap on the device
+ *                must not share it.
+ *   status       optional device int32 (ORTHRUS_STATUS_TIMEOUT only).
+ *
+ * Supported: B * K <= ORTHRUS_MAX_LM_ROWS, Hd a multiple of 64, V < 2^31;
+ * hidden, lm_head and workspace 16-byte aligned; sm_100 devices only.
+ * Numerics: logits are fp32 sums of exact bf16 products; an argmax whose top
+ * two logits differ by less than the fp32 rounding of the row can differ from
+ * an exact (fp64) evaluation.
+ */
+ORTHRUS_API int orthrus_lm_head_consensus(const void *hidden, const void *lm_head,
+                                          const int32_t *proposed, int B, int K, int V, int Hd,
+                                          int32_t *accepted_len, int32_t *next_token,
+                                          int32_t *argmax_out, void *workspace,
+                                          size_t workspace_bytes, int32_t *status, void *stream);
+
 /* Human-readable text for an ORTHRUS_* return code (static storage). */
 ORTHRUS_API const char *orthrus_error_string(int code);
 

@@ -24,7 +24,8 @@ STATUS_CAPACITY, STATUS_ACCEPT, STATUS_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn", "orthrus_attn_path",
             "orthrus_consensus_workspace_size", "orthrus_consensus",
             "orthrus_kv_commit", "orthrus_write_block", "orthrus_error_string",
-            "orthrus_version")
+            "orthrus_version", "orthrus_lm_head_workspace_size",
+            "orthrus_lm_head_consensus")
 
 
 class OrthrusError(RuntimeError):
@@ -63,6 +64,11 @@ def lib():
                                           i32, vp, vp]
         L.orthrus_attn_path.restype = i32
         L.orthrus_attn_path.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.orthrus_lm_head_workspace_size.restype = sz
+        L.orthrus_lm_head_workspace_size.argtypes = [i32, i32]
+        L.orthrus_lm_head_consensus.restype = i32
+        L.orthrus_lm_head_consensus.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz,
+                                                vp, vp]
         L.orthrus_error_string.restype = ctypes.c_char_p
         L.orthrus_error_string.argtypes = [i32]
         L.orthrus_version.restype = i32
@@ -190,3 +196,24 @@ def orthrus_kv_commit(ctx_lens: torch.Tensor, accepted_len: torch.Tensor, *, K: 
                                  _ptr(ctx_lens), _ptr(accepted_len), B, Hkv, D, S_max, K,
                                  _dtype_code(dtype), _ptr(status), _stream(stream))
     _check("orthrus_kv_commit", rc)
+
+
+def orthrus_lm_head_workspace_size(B: int, K: int) -> int:
+    return int(lib().orthrus_lm_head_workspace_size(B, K))
+
+
+def orthrus_lm_head_consensus(hidden: torch.Tensor, lm_head: torch.Tensor, proposed: torch.Tensor,
+                              accepted_len: torch.Tensor, next_token: torch.Tensor,
+                              workspace: torch.Tensor, argmax_out: Optional[torch.Tensor] = None,
+                              status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """hidden [B,K,Hd] bf16, lm_head [V,Hd] bf16, proposed [B,K] int32 ->
+    accepted_len [B], next_token [B] (the logits are never materialised)."""
+    B, K, Hd = hidden.shape
+    V = lm_head.shape[0]
+    assert hidden.dtype == torch.bfloat16 and lm_head.dtype == torch.bfloat16
+    assert proposed.dtype == torch.int32 and lm_head.shape[1] == Hd
+    rc = lib().orthrus_lm_head_consensus(_ptr(hidden), _ptr(lm_head), _ptr(proposed), B, K, V, Hd,
+                                         _ptr(accepted_len), _ptr(next_token), _ptr(argmax_out),
+                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _ptr(status), _stream(stream))
+    _check("orthrus_lm_head_consensus", rc)

@@ -87,6 +87,21 @@ struct ConsensusArgs {
 };
 cudaError_t launch_consensus(const ConsensusArgs &p, cudaStream_t st);
 
+// Fused AR LM head + argmax + consensus (lm_head.cu).
+constexpr int kMaxLmRows = ORTHRUS_MAX_LM_ROWS;   // B * K token rows per call
+struct LmHeadArgs {
+    const int32_t *proposed;
+    int32_t *accepted;
+    int32_t *next_token;
+    int32_t *argmax_out;
+    unsigned long long *ws_keys;         // [B*K] packed (value, index) maxima, zero between calls
+    unsigned int *ws_done;               // CTAs finished, zero between calls
+    int32_t *status;
+    int B, K, V, Hd;
+    int Np;                              // token rows padded for the MMA's N
+    int nst;                             // pipeline stages
+};
+
 struct CommitArgs {
     void *k_caches[ORTHRUS_MAX_LAYERS];
     void *v_caches[ORTHRUS_MAX_LAYERS];

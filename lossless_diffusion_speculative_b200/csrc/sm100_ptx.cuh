@@ -72,7 +72,7 @@ __device__ __forceinline__ unsigned long long global_ns()
 
 // Bounded wait: false when the CTA aborted or this wait ran out of time (the
 // latter raises ORTHRUS_STATUS_TIMEOUT and sets the CTA's abort flag).
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+static __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                       int32_t *status)
 {
     if (mbar_try(bar, parity)) return true;
@@ -91,7 +91,7 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile in
 }
 
 // Drain wait used on the abort path: bounded, no side effects.
-__device__ __noinline__ void wait_bar_quiet(uint32_t bar, uint32_t parity)
+static __device__ __noinline__ void wait_bar_quiet(uint32_t bar, uint32_t parity)
 {
     const unsigned long long t0 = global_ns();
     while (!mbar_try(bar, parity))
@@ -101,6 +101,15 @@ __device__ __noinline__ void wait_bar_quiet(uint32_t bar, uint32_t parity)
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)m) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"((unsigned long long)m), "r"(bar), "r"(x), "r"(y)
+        : "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, uint32_t bar,

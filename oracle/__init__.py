@@ -214,3 +214,71 @@ def fp32_dot_error_bound(n: int, absdot) -> np.ndarray:
     """
     u = 2.0 ** -23
     return n * u / (1.0 - n * u) * np.asarray(absdot, np.float64)
+
+
+def _softmax64(x: np.ndarray, temperature: float) -> np.ndarray:
+    z = np.asarray(x, np.float64) / float(temperature)
+    z = z - z.max()
+    e = np.exp(z)
+    return e / e.sum()
+
+
+def rejection_verify(ar_logits: np.ndarray, draft_logits: np.ndarray, proposed: np.ndarray,
+                     u_accept: np.ndarray, u_resample: np.ndarray, temperature: float):
+    """Lossless verification of the block at temperature T > 0 (the pages
+    evaluate "greedy and rejection sampling" -- Orthrus-Qwen3, agentlenshq.com,
+    "limitations"; results "depending on task and temperature" -- gist.science
+    technical summary, section 4 -- without a formula; this is the standard
+    speculative-sampling rule, which keeps the AR head's distribution exactly).
+
+    For sequence b, left to right over block slots i, with p = softmax(AR
+    logits / T) and q = softmax(draft logits / T) of row i and x = proposed[b, i]:
+      accept x  iff  u_accept[b, i] * q(x) < p(x)      (probability min(1, p/q));
+    at the first rejection (slot a) the next token is drawn from the residual
+    r(v) = max(0, p(v) - q(v)) by inverse CDF: the smallest v whose cumulative
+    residual exceeds u_resample[b] * sum_v r(v) (from p itself if the residual
+    is empty).  With all K accepted the next token is the last proposal (the AR
+    view has not scored a token after the block).  Everything in float64.
+
+    Returns (accepted [B], next [B], acc_margin [B, K], cdf_margin [B]): the
+    relative margin of every accept decision taken, |u q(x) - p(x)| /
+    max(p(x), u q(x)) (inf where not taken), and the distance of the resampling
+    target from the nearest cumulative-residual boundary relative to the total
+    residual (inf when nothing was resampled).
+    """
+    B, K, V = ar_logits.shape
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    acc_margin = np.full((B, K), np.inf)
+    cdf_margin = np.full(B, np.inf)
+    for b in range(B):
+        a = 0
+        p = q = None
+        while a < K:
+            p = _softmax64(ar_logits[b, a], temperature)
+            q = _softmax64(draft_logits[b, a], temperature)
+            x = int(proposed[b, a])
+            lhs = float(u_accept[b, a]) * q[x]
+            den = max(p[x], lhs)
+            acc_margin[b, a] = abs(lhs - p[x]) / den if den > 0 else np.inf
+            if not lhs < p[x]:
+                break
+            a += 1
+        acc[b] = a
+        if a == K:
+            nxt[b] = int(proposed[b, K - 1])
+            continue
+        r = np.maximum(p - q, 0.0)
+        if r.sum() <= 0.0:
+            r = p
+        cdf = np.cumsum(r)
+        R = cdf[-1]
+        target = float(u_resample[b]) * R
+        v = int(np.searchsorted(cdf, target, side="right"))
+        v = min(v, V - 1)
+        while v > 0 and r[v] == 0.0:                  # (a zero-mass tail is never drawn)
+            v -= 1
+        nxt[b] = v
+        lo = cdf[v - 1] if v > 0 else 0.0
+        cdf_margin[b] = min(target - lo, cdf[v] - target) / R
+    return acc, nxt, acc_margin, cdf_margin

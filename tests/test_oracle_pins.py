@@ -455,3 +455,66 @@ def test_fp32_accumulation_stays_within_the_stated_bound():
                 acc = np.float32(acc + v)
             assert abs(float(acc) - exact) <= bound
         assert abs(float(np.sum(p32, dtype=np.float32)) - exact) <= bound
+
+
+# --------------------------------------------------------------------------- rejection sampling
+
+def test_rejection_is_lossless_monte_carlo():
+    """Proposals drawn from q, verified against p: the emitted token of a
+    one-slot block is distributed as p (chi-square over 6 tokens)."""
+    rng = np.random.default_rng(50)
+    V, N, T = 6, 60000, 0.8
+    ar = rng.standard_normal(V) * 1.5
+    dr = rng.standard_normal(V) * 1.5
+    p = np.exp(ar / T) / np.exp(ar / T).sum()
+    q = np.exp(dr / T) / np.exp(dr / T).sum()
+    x = rng.choice(V, size=N, p=q).astype(np.int32)
+    acc, nxt, _, _ = oracle.rejection_verify(np.broadcast_to(ar, (N, 1, V)), np.broadcast_to(dr, (N, 1, V)),
+                                             x[:, None], rng.random((N, 1)), rng.random(N), T)
+    emitted = np.where(acc == 1, x, nxt)
+    counts = np.bincount(emitted, minlength=V)
+    chi2 = float((((counts - N * p) ** 2) / (N * p)).sum())
+    assert chi2 < 30.0, (chi2, counts, N * p)          # 5 dof: P(chi2 > 30) ~ 1.5e-5
+
+
+def test_rejection_at_low_temperature_is_greedy():
+    """T -> 0 with argmax-q proposals: the rule reduces to the greedy
+    consensus (the independent C oracle) on the AR logits."""
+    w = wl.WORKLOADS["qwen3_4b_ragged"].with_(B=4, K=8, vocab=300)
+    ci = wl.consensus_inputs(w)
+    rng = np.random.default_rng(51)
+    draft = rng.standard_normal(ci.logits.shape).astype(np.float32)
+    draft[np.arange(4)[:, None], np.arange(8)[None, :], ci.proposed] += 20.0   # q peaks at the proposal
+    acc, nxt, _, _ = oracle.rejection_verify(ci.logits, draft, ci.proposed, rng.random((4, 8)),
+                                             rng.random(4), 1e-3)
+    gacc, gnxt, _ = oracle.consensus(ci.logits, ci.proposed)
+    assert (acc == gacc).all() and (nxt == gnxt).all()
+
+
+def test_rejection_identical_views_accept_everything():
+    rng = np.random.default_rng(52)
+    lg = rng.standard_normal((3, 5, 40))
+    prop = rng.integers(0, 40, (3, 5)).astype(np.int32)
+    acc, nxt, _, _ = oracle.rejection_verify(lg, lg, prop, rng.random((3, 5)) * 0.999, rng.random(3), 1.3)
+    assert (acc == 5).all() and (nxt == prop[:, 4]).all()
+
+
+def test_rejection_hand_cases():
+    """p = (.5, .3, .2), q = (.2, .3, .5) at T = 1: x = 2 is kept with
+    probability .4 and the residual (.3, 0, 0) always yields token 0; x = 0
+    (ratio 2.5) is always kept.  A two-token residual splits at its midpoint."""
+    ar = np.log(np.array([[[0.5, 0.3, 0.2]]]))
+    dr = np.log(np.array([[[0.2, 0.3, 0.5]]]))
+    for u, a, n in ((0.5, 0, 0), (0.3, 1, 2), (0.399, 1, 2), (0.401, 0, 0)):
+        acc, nxt, _, _ = oracle.rejection_verify(ar, dr, np.array([[2]], np.int32), np.array([[u]]),
+                                                 np.array([0.77]), 1.0)
+        assert (acc[0], nxt[0]) == (a, n), (u, acc, nxt)
+    acc, _, _, _ = oracle.rejection_verify(ar, dr, np.array([[0]], np.int32), np.array([[0.999]]),
+                                           np.array([0.5]), 1.0)
+    assert acc[0] == 1
+    ar2 = np.log(np.array([[[0.5, 0.5, 1e-12]]]))
+    dr2 = np.log(np.array([[[0.1, 0.1, 0.8]]]))            # residual (.4, .4, 0)
+    for up, n in ((0.3, 0), (0.6, 1), (0.49, 0), (0.51, 1)):
+        acc, nxt, _, cm = oracle.rejection_verify(ar2, dr2, np.array([[2]], np.int32), np.array([[0.9]]),
+                                                  np.array([up]), 1.0)
+        assert acc[0] == 0 and nxt[0] == n, (up, nxt)
