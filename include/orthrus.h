@@ -182,6 +182,50 @@ ORTHRUS_API int orthrus_consensus(const float *logits, const int32_t *proposed, 
                       size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
+ * orthrus_rejection_workspace_size — scratch bytes for orthrus_rejection_verify
+ * (one 16-byte (max, sum) pair of both views per vocabulary chunk per row).
+ */
+ORTHRUS_API size_t orthrus_rejection_workspace_size(int B, int K, int V);
+
+/*
+ * orthrus_rejection_verify — lossless verification at temperature T > 0, the
+ * sampling counterpart of orthrus_consensus (the pages evaluate greedy and
+ * rejection-sampling decoding -- Orthrus-Qwen3, agentlenshq.com blog,
+ * "limitations"; gist.science technical summary, section 4 -- without giving
+ * the rule; this is the standard speculative-sampling rule, which leaves the
+ * AR head's distribution unchanged).
+ *
+ * For sequence b, left to right over block slots i, with p = softmax(
+ * ar_logits[b, i, :] / T), q = softmax(draft_logits[b, i, :] / T) and x =
+ * proposed[b, i]:
+ *     x is kept  iff  u_accept[b, i] * q(x) < p(x)   (probability min(1, p/q));
+ * a proposal outside [0, V) is never kept.  accepted_len[b] = number of leading
+ * slots kept, in [0, K].  At the first rejection a, next_token[b] is drawn from
+ * the residual r(v) = max(0, p(v) - q(v)) by inverse CDF: the smallest v whose
+ * cumulative residual exceeds u_resample[b] * sum_v r(v) (from p itself when the
+ * residual is empty).  With all K kept, next_token[b] = proposed[b, K - 1]
+ * (the AR view has not scored a token after the block).
+ *
+ *   ar_logits, draft_logits  [B, K, V] fp32, finite; 16-byte aligned.
+ *   proposed     [B, K] int32 (drawn by the caller from q).
+ *   u_accept     [B, K] fp32 uniform draws in [0, 1) (the caller's generator).
+ *   u_resample   [B] fp32 uniform draws in [0, 1).
+ *   temperature  > 0.
+ *   workspace    >= orthrus_rejection_workspace_size(B, K, V) bytes, 16-byte
+ *                aligned, clobbered.
+ * Supported: K <= ORTHRUS_MAX_BLOCK, V <= 262144, B * K <= 65535.
+ * Numerics: fp32 with exp2 on the special-function unit; a decision whose
+ * margin is within ~1e-6 relative of its threshold can differ from an exact
+ * evaluation.
+ */
+ORTHRUS_API int orthrus_rejection_verify(const float *ar_logits, const float *draft_logits,
+                                         const int32_t *proposed, const float *u_accept,
+                                         const float *u_resample, float temperature, int B,
+                                         int K, int V, int32_t *accepted_len, int32_t *next_token,
+                                         void *workspace, size_t workspace_bytes, int32_t *status,
+                                         void *stream);
+
+/*
  * orthrus_kv_commit — commit the accepted prefix of the block for every layer
  * and advance the committed length once (section 2.3: commit the synchronised
  * prefix and truncate the cache; rollback is a length change, no data moves).

@@ -25,7 +25,8 @@ EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn", "orthrus_attn_path",
             "orthrus_consensus_workspace_size", "orthrus_consensus",
             "orthrus_kv_commit", "orthrus_write_block", "orthrus_error_string",
             "orthrus_version", "orthrus_lm_head_workspace_size",
-            "orthrus_lm_head_consensus")
+            "orthrus_lm_head_consensus", "orthrus_rejection_workspace_size",
+            "orthrus_rejection_verify")
 
 
 class OrthrusError(RuntimeError):
@@ -69,6 +70,11 @@ def lib():
         L.orthrus_lm_head_consensus.restype = i32
         L.orthrus_lm_head_consensus.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz,
                                                 vp, vp]
+        L.orthrus_rejection_workspace_size.restype = sz
+        L.orthrus_rejection_workspace_size.argtypes = [i32, i32, i32]
+        L.orthrus_rejection_verify.restype = i32
+        L.orthrus_rejection_verify.argtypes = [vp, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, vp, sz,
+                                               vp, vp]
         L.orthrus_error_string.restype = ctypes.c_char_p
         L.orthrus_error_string.argtypes = [i32]
         L.orthrus_version.restype = i32
@@ -217,3 +223,26 @@ def orthrus_lm_head_consensus(hidden: torch.Tensor, lm_head: torch.Tensor, propo
                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
                                          _ptr(status), _stream(stream))
     _check("orthrus_lm_head_consensus", rc)
+
+
+def orthrus_rejection_workspace_size(B: int, K: int, V: int) -> int:
+    return int(lib().orthrus_rejection_workspace_size(B, K, V))
+
+
+def orthrus_rejection_verify(ar_logits: torch.Tensor, draft_logits: torch.Tensor,
+                             proposed: torch.Tensor, u_accept: torch.Tensor, u_resample: torch.Tensor,
+                             temperature: float, accepted_len: torch.Tensor, next_token: torch.Tensor,
+                             workspace: torch.Tensor, status: Optional[torch.Tensor] = None,
+                             stream=None) -> None:
+    """Logits [B,K,V] fp32 of both views, proposals [B,K] int32, uniform draws
+    u_accept [B,K] and u_resample [B] fp32 -> accepted_len [B], next_token [B]."""
+    B, K, V = ar_logits.shape
+    assert ar_logits.dtype == torch.float32 and draft_logits.dtype == torch.float32
+    assert draft_logits.shape == ar_logits.shape and proposed.dtype == torch.int32
+    assert u_accept.dtype == torch.float32 and u_resample.dtype == torch.float32
+    rc = lib().orthrus_rejection_verify(_ptr(ar_logits), _ptr(draft_logits), _ptr(proposed),
+                                        _ptr(u_accept), _ptr(u_resample), float(temperature), B, K, V,
+                                        _ptr(accepted_len), _ptr(next_token), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _ptr(status),
+                                        _stream(stream))
+    _check("orthrus_rejection_verify", rc)

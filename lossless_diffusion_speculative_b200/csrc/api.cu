@@ -202,6 +202,52 @@ int orthrus_consensus(const float *logits, const int32_t *proposed, int B, int K
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 
+size_t orthrus_rejection_workspace_size(int B, int K, int V)
+{
+    if (B <= 0 || K <= 0 || V <= 0 || K > ORTHRUS_MAX_BLOCK) return 0;
+    const int sms = current_sm_count();
+    if (sms <= 0) return 0;
+    int s, c;
+    consensus_split(B, K, V, sms, &s, &c);
+    return (size_t)B * K * s * sizeof(float4);
+}
+
+int orthrus_rejection_verify(const float *ar_logits, const float *draft_logits, const int32_t *proposed,
+                             const float *u_accept, const float *u_resample, float temperature, int B,
+                             int K, int V, int32_t *accepted_len, int32_t *next_token, void *workspace,
+                             size_t workspace_bytes, int32_t *status, void *stream)
+{
+    if (!ar_logits || !draft_logits || !proposed || !u_accept || !u_resample || !accepted_len ||
+        !next_token)
+        return ORTHRUS_ERR_ARG;
+    if (B <= 0 || K <= 0 || V <= 0 || !(temperature > 0.f) || isinf(temperature)) return ORTHRUS_ERR_ARG;
+    if (K > ORTHRUS_MAX_BLOCK || V > kMaxRejectTiles * 128 || (int64_t)B * K > 65535)
+        return ORTHRUS_ERR_UNSUPPORTED;
+    if (!aligned16(ar_logits) || !aligned16(draft_logits) || (workspace && !aligned16(workspace)))
+        return ORTHRUS_ERR_ALIGN;
+    const int sms = current_sm_count();
+    if (sms <= 0) return ORTHRUS_ERR_DEVICE;
+    RejectArgs a;
+    consensus_split(B, K, V, sms, &a.splits, &a.chunk);
+    const size_t need = (size_t)B * K * a.splits * sizeof(float4);
+    if (!workspace || workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+    a.ar = ar_logits;
+    a.dr = draft_logits;
+    a.proposed = proposed;
+    a.u_accept = u_accept;
+    a.u_resample = u_resample;
+    a.accepted = accepted_len;
+    a.next_token = next_token;
+    a.ws = static_cast<float4 *>(workspace);
+    a.status = status;
+    a.B = B;
+    a.K = K;
+    a.V = V;
+    a.c = kLog2e / temperature;
+    const cudaError_t e = launch_rejection(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
 static int fill_layer_ptrs(CommitArgs &a, int num_layers, void *const *k_caches,
                            void *const *v_caches, const void *const *k_blks,
                            const void *const *v_blks, int D)

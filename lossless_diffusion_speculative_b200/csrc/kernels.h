@@ -100,7 +100,24 @@ struct LmHeadArgs {
     int B, K, V, Hd;
     int Np;                              // token rows padded for the MMA's N
     int nst;                             // pipeline stages
+    int cps;                             // adjacent 64-wide hidden chunks per stage
 };
+
+// Rejection-sampling verification (rejection.cu).
+constexpr int kMaxRejectTiles = 2048;    // vocabulary <= 2048 * 128 = 262144
+struct RejectArgs {
+    const float *ar, *dr;                // [B*K, V] AR-view and draft-view logits
+    const int32_t *proposed;             // [B*K]
+    const float *u_accept;               // [B*K] uniform draws in [0, 1)
+    const float *u_resample;             // [B]
+    int32_t *accepted;
+    int32_t *next_token;
+    float4 *ws;                          // [B*K, splits] (max, sum) of both views, log2 units
+    int32_t *status;
+    int B, K, V, splits, chunk;
+    float c;                             // log2(e) / temperature
+};
+cudaError_t launch_rejection(const RejectArgs &p, cudaStream_t st);
 
 struct CommitArgs {
     void *k_caches[ORTHRUS_MAX_LAYERS];

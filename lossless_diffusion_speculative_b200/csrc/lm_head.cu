@@ -41,7 +41,8 @@ using namespace sm100;
 
 constexpr int kThreads = 192;
 constexpr int kTileRows = 128;
-constexpr int kChunk = 64;                         // hidden dims per stage (128 bytes of bf16)
+constexpr int kChunk = 64;                         // hidden dims per box (128 bytes of bf16)
+
 constexpr uint32_t kABytes = kTileRows * 128;      // 16 KiB
 constexpr int kMaxStages = 12;
 constexpr uint32_t kRingBudget = 200 * 1024;
@@ -62,10 +63,13 @@ struct Layout {
     uint32_t stage_bytes, ring, bars, misc, keys, rbuf, total;
 };
 
-__host__ __device__ inline Layout layout_of(int Np, int nst)
+// A pipeline stage holds `cps` adjacent hidden chunks: every weight row then
+// gives cps * 128 contiguous bytes per stage, which the memory system serves
+// far better than 128-byte pieces 8 KiB apart (weight rows are Hd * 2 bytes).
+__host__ __device__ inline Layout layout_of(int Np, int nst, int cps)
 {
     Layout l;
-    l.stage_bytes = kABytes + (uint32_t)Np * 128u;
+    l.stage_bytes = (uint32_t)cps * (kABytes + (uint32_t)Np * 128u);
     l.ring = 0;
     l.bars = (uint32_t)nst * l.stage_bytes;
     l.misc = l.bars + B_COUNT * 8;
@@ -126,7 +130,8 @@ struct Smem {
     volatile int *abort_flag;
     __device__ __forceinline__ uint32_t bar(int i) const { return base + L.bars + 8u * i; }
     __device__ __forceinline__ uint32_t a_of(int st) const { return base + st * L.stage_bytes; }
-    __device__ __forceinline__ uint32_t b_of(int st) const { return a_of(st) + kABytes; }
+    int cps;
+    __device__ __forceinline__ uint32_t b_of(int st) const { return a_of(st) + cps * kABytes; }
 };
 
 // The CTA's vocabulary rows [lo, hi) and tile count.
@@ -146,12 +151,16 @@ __device__ __forceinline__ Range range_of(int V, int cid, int grid)
     return rg;
 }
 
+template <int CPS>
 __device__ __forceinline__ void producer(const Smem &sh, const LmHeadArgs &p, const Range &rg,
                                          const CUtensorMap *tw, const CUtensorMap *tw16,
                                          const CUtensorMap *th)
 {
     const int nk = p.Hd / kChunk;
     const int half = p.Np > 256 ? p.Np / 2 : p.Np;
+    // (every CTA sweeps the hidden dimension in the same order, so equal weight
+    // rows give bit-equal logits and exact ties resolve to the lower index)
+    const uint64_t pol_w = make_policy_evict_first(), pol_h = make_policy_evict_last();
     uint32_t it = 0;
     bool ok = true;
     for (int t = 0; t < rg.ntile && ok; ++t) {
@@ -159,7 +168,7 @@ __device__ __forceinline__ void producer(const Smem &sh, const LmHeadArgs &p, co
         const int nrows = rg.hi - r0 < kTileRows ? rg.hi - r0 : kTileRows;
         const int nb16 = (nrows + 15) >> 4;
         const uint32_t a_bytes = nrows == kTileRows ? kABytes : (uint32_t)nb16 * 16u * 128u;
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+        for (int ks = 0; ks < nk / CPS; ++ks, ++it) {
             const int st = it % p.nst;
             const uint32_t n = it / p.nst;
             if (n > 0 && !wait_bar(sh.bar(B_EMPTY + st), (n - 1) & 1, sh.abort_flag, p.status)) {
@@ -167,14 +176,22 @@ __device__ __forceinline__ void producer(const Smem &sh, const LmHeadArgs &p, co
                 break;
             }
             const uint32_t full = sh.bar(B_FULL + st);
-            mbar_expect_tx(full, a_bytes + (uint32_t)p.Np * 128u);
-            if (nrows == kTileRows) {
-                tma_load_2d(sh.a_of(st), tw, full, kc * kChunk, r0);
-            } else {
-                for (int j = 0; j < nb16; ++j) tma_load_2d(sh.a_of(st) + j * 2048u, tw16, full, kc * kChunk, r0 + 16 * j);
+            mbar_expect_tx(full, CPS * (a_bytes + (uint32_t)p.Np * 128u));
+            // (the stage's chunks are adjacent in every weight row: issued back to back)
+#pragma unroll
+            for (int j = 0; j < CPS; ++j) {
+                const int kc = ks * CPS + j;
+                const uint32_t a = sh.a_of(st) + j * kABytes;
+                if (nrows == kTileRows) {
+                    tma_load_2d_hint(a, tw, full, kc * kChunk, r0, pol_w);
+                } else {
+                    for (int q = 0; q < nb16; ++q)
+                        tma_load_2d_hint(a + q * 2048u, tw16, full, kc * kChunk, r0 + 16 * q, pol_w);
+                }
+                const uint32_t b = sh.b_of(st) + j * (uint32_t)p.Np * 128u;
+                tma_load_2d_hint(b, th, full, kc * kChunk, 0, pol_h);
+                if (half != p.Np) tma_load_2d_hint(b + (uint32_t)half * 128u, th, full, kc * kChunk, half, pol_h);
             }
-            tma_load_2d(sh.b_of(st), th, full, kc * kChunk, 0);
-            if (half != p.Np) tma_load_2d(sh.b_of(st) + (uint32_t)half * 128u, th, full, kc * kChunk, half);
         }
     }
     if (!ok) {                       // abort: let every copy already issued land
@@ -185,6 +202,7 @@ __device__ __forceinline__ void producer(const Smem &sh, const LmHeadArgs &p, co
     }
 }
 
+template <int CPS>
 __device__ __forceinline__ void mma_issuer(const Smem &sh, const LmHeadArgs &p, const Range &rg, uint32_t tmem)
 {
     const int nk = p.Hd / kChunk;
@@ -202,21 +220,25 @@ __device__ __forceinline__ void mma_issuer(const Smem &sh, const LmHeadArgs &p, 
         }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * p.Np);
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+        for (int ks = 0; ks < nk / CPS; ++ks, ++it) {
             const int st = it % p.nst;
             if (!wait_bar(sh.bar(B_FULL + st), (it / p.nst) & 1, sh.abort_flag, p.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint64_t ad = smem_desc(sh.a_of(st), 16, 1024);
-            const uint64_t bd = smem_desc(sh.b_of(st), 16, 1024);
-            const uint64_t bd2 = smem_desc(sh.b_of(st) + (uint32_t)n_mma * 128u, 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {            // 16 hidden dims (32 bytes) per MMA
-                const uint32_t on = (kc | kk) ? 1u : 0u;
-                tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, on);
-                if (split) tc_mma_ss(d + (uint32_t)n_mma, ad + 2 * kk, bd2 + 2 * kk, idesc, on);
+            for (int j = 0; j < CPS; ++j) {
+                const uint32_t b = sh.b_of(st) + j * (uint32_t)p.Np * 128u;
+                const uint64_t ad = smem_desc(sh.a_of(st) + j * kABytes, 16, 1024);
+                const uint64_t bd = smem_desc(b, 16, 1024);
+                const uint64_t bd2 = smem_desc(b + (uint32_t)n_mma * 128u, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {        // 16 hidden dims (32 bytes) per MMA
+                    const uint32_t on = (ks | j | kk) ? 1u : 0u;
+                    tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, on);
+                    if (split) tc_mma_ss(d + (uint32_t)n_mma, ad + 2 * kk, bd2 + 2 * kk, idesc, on);
+                }
             }
             tc_commit(sh.bar(B_EMPTY + st));
         }
@@ -260,6 +282,7 @@ __device__ __forceinline__ bool epilogue(const Smem &sh, const LmHeadArgs &p, co
     return true;
 }
 
+template <int CPS>
 __global__ void __launch_bounds__(kThreads, 1)
     lm_head_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_w16,
                    const __grid_constant__ CUtensorMap tm_h, const LmHeadArgs p)
@@ -270,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem sh;
     sh.base = aligned;
     sh.ptr = smem_raw + (aligned - raw);
-    sh.L = layout_of(p.Np, p.nst);
+    sh.L = layout_of(p.Np, p.nst, p.cps);
+    sh.cps = p.cps;
     sh.abort_flag = reinterpret_cast<volatile int *>(sh.ptr + sh.L.misc + 4);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sh.ptr + sh.L.misc);
     volatile int *last_flag = reinterpret_cast<volatile int *>(sh.ptr + sh.L.misc + 8);
@@ -319,10 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4) {
         epilogue(sh, p, rg, tmem);                 // (an abort sets the CTA's abort flag)
     } else if (warp == 4) {
-        if (lane == 0) producer(sh, p, rg, &tm_w, &tm_w16, &tm_h);
+        if (lane == 0) producer<CPS>(sh, p, rg, &tm_w, &tm_w16, &tm_h);
         __syncwarp();
     } else {
-        if (lane == 0) mma_issuer(sh, p, rg, tmem);
+        if (lane == 0) mma_issuer<CPS>(sh, p, rg, tmem);
         __syncwarp();
     }
     tc_fence_before();
@@ -382,18 +406,34 @@ bool lm_smem_ready(int dev)
 {
     if (dev < 0 || dev >= kMaxDevices) return false;
     std::call_once(g_smem_once[dev], [dev] {
-        g_smem_ok[dev] = cudaFuncSetAttribute(lmh::lm_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              227 * 1024) == cudaSuccess;
+        const int lim = 227 * 1024;
+        g_smem_ok[dev] =
+            cudaFuncSetAttribute(lmh::lm_head_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(lmh::lm_head_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(lmh::lm_head_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess;
         if (!g_smem_ok[dev]) cudaGetLastError();
     });
     return g_smem_ok[dev];
 }
 
-int lm_stages(int Np)
+// Chunks per stage: the most (4, 2 or 1) that divide the hidden size and
+// still leave two stages in the ring; then as many stages as fit.
+void lm_pipeline(int Np, int nk, int *cps, int *nst)
 {
-    const uint32_t sb = lmh::kABytes + (uint32_t)Np * 128u;
-    int n = (int)(lmh::kRingBudget / sb);
-    return n > lmh::kMaxStages ? lmh::kMaxStages : n;
+    *cps = 1;
+    for (int c = 4; c >= 2; c >>= 1) {
+        const uint32_t sb = (uint32_t)c * (lmh::kABytes + (uint32_t)Np * 128u);
+        if (nk % c == 0 && 2 * sb <= lmh::kRingBudget) {
+            *cps = c;
+            break;
+        }
+    }
+    const uint32_t sb = (uint32_t)*cps * (lmh::kABytes + (uint32_t)Np * 128u);
+    const int n = (int)(lmh::kRingBudget / sb);
+    *nst = n > lmh::kMaxStages ? lmh::kMaxStages : n;
 }
 
 }  // namespace
@@ -445,8 +485,8 @@ int orthrus_lm_head_consensus(const void *hidden, const void *lm_head, const int
     a.V = V;
     a.Hd = Hd;
     a.Np = Np;
-    a.nst = lm_stages(Np);
-    const lmh::Layout L = lmh::layout_of(Np, a.nst);
+    lm_pipeline(Np, Hd / 64, &a.cps, &a.nst);
+    const lmh::Layout L = lmh::layout_of(Np, a.nst, a.cps);
 
     CUtensorMap tw, tw16, th;
     const uint64_t wdims[2] = {(uint64_t)Hd, (uint64_t)V}, wstr[1] = {(uint64_t)Hd * 2};
@@ -469,7 +509,9 @@ int orthrus_lm_head_consensus(const void *hidden, const void *lm_head, const int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel, tw, tw16, th, a);
+    const cudaError_t e = a.cps == 4   ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<4>, tw, tw16, th, a)
+                          : a.cps == 2 ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<2>, tw, tw16, th, a)
+                                       : cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<1>, tw, tw16, th, a);
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 

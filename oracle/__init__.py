@@ -282,3 +282,14 @@ def rejection_verify(ar_logits: np.ndarray, draft_logits: np.ndarray, proposed: 
         lo = cdf[v - 1] if v > 0 else 0.0
         cdf_margin[b] = min(target - lo, cdf[v] - target) / R
     return acc, nxt, acc_margin, cdf_margin
+
+
+def residual_cdf(ar_row: np.ndarray, draft_row: np.ndarray, temperature: float) -> np.ndarray:
+    """float64 cumulative residual max(0, p - q) of one row (of p itself when
+    the residual is empty), the distribution rejection_verify draws from."""
+    p = _softmax64(ar_row, temperature)
+    q = _softmax64(draft_row, temperature)
+    r = np.maximum(p - q, 0.0)
+    if r.sum() <= 0.0:
+        r = p
+    return np.cumsum(r)
