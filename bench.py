@@ -311,6 +311,60 @@ def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
     return out
 
 
+# ----------------------------------------------------------------------------- fused layer step
+def measure_fused_step(name, dev, stream, hbm, iters, st=None):
+    """The decode step with each layer's QKV projection fused with the cache
+    tail write (orthrus_qkv_project) ahead of its attention, per view, then
+    consensus and commit: the fused step's median µs, and the projections
+    alone (same launches, no attention) for their weight-read bandwidth."""
+    import torch
+    from lossless_diffusion_speculative_b200 import workloads as wl
+    from lossless_diffusion_speculative_b200.step import DecodeStep
+
+    w = wl.WORKLOADS[name]
+    if st is None:
+        st = DecodeStep(w, order="fused", device=dev, project=True)
+    else:
+        st.enable_projection()
+    out = {"workload": name, "layers": st.L, "B": w.B, "K": w.K, "hidden": w.hidden}
+    for order in ("fused", "project_only"):
+        graphs = st.capture(stream, order=order)
+        names = [n for n, _ in graphs[1:]]
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in names] for _ in range(iters)]
+        with torch.cuda.stream(stream):
+            for it in range(3 + iters):
+                graphs[0][1].replay()
+                for k, (_, g) in enumerate(graphs[1:]):
+                    if it >= 3:
+                        ev[it - 3][k][0].record()
+                    g.replay()
+                    if it >= 3:
+                        ev[it - 3][k][1].record()
+            torch.cuda.synchronize()
+        if int(st.status.item()) != 0:
+            raise RuntimeError(f"fused step {name}: device status {int(st.status.item()):#x}")
+        med = {n: float(np.median([ev[i][k][0].elapsed_time(ev[i][k][1]) for i in range(iters)])) * 1e3
+               for k, n in enumerate(names)}
+        out["segments_us_" + order] = med
+        del graphs
+    fused = out["segments_us_fused"]
+    proj = out["segments_us_project_only"]
+    step_us = sum(fused.values())
+    proj_us = sum(proj.values())
+    calls = 2 * st.L
+    wbytes = sum(t.numel() * t.element_size() for t in st.w_qkv[0])
+    out.update({"step_us": step_us, "project_us_per_call": proj_us / calls,
+                "project_weight_bytes": wbytes,
+                "project_weight_read_gbs": wbytes / (proj_us / calls * 1e-6) / 1e9,
+                "project_frac_of_hbm": wbytes / (proj_us / calls * 1e-6) / 1e9 / hbm,
+                "attn_us_in_step_est": step_us - fused.get("consensus_commit", 0.0) - proj_us,
+                "verified_tokens_per_s": st.tokens_per_step() / (step_us * 1e-6),
+                "verified_tokens_per_s_at_expected": st.tokens_per_step_expected() / (step_us * 1e-6),
+                "timing": "median of per-segment CUDA events over graph replays (inputs larger than L2)"})
+    return out
+
+
 # ----------------------------------------------------------------------------- fused LM head
 LM_HEAD_SET = ("qwen3_1p7b_layer", "qwen3_8b_step", "qwen3_4b_ragged", "qwen3_8b_long_k32")
 
@@ -372,6 +426,56 @@ def measure_lm_head(name, dev, stream, hbm, iters):
            "kernel": "lm_head_kernel (tcgen05 swap-AB GEMM, argmax epilogue, last-CTA consensus)",
            "timing": "median of CUDA events per call; L2 flushed before each call"}
     del W, h, flush
+    return out
+
+
+# ----------------------------------------------------------------------------- rejection sampling
+REJECT_SET = ("qwen3_8b_step", "qwen3_4b_ragged", "qwen3_8b_long_k32")
+
+
+def measure_rejection(name, dev, stream, hbm, iters):
+    """orthrus_rejection_verify (temperature 1) on the workload's [B, K, V]
+    logits of both views: median µs per call, L2 flushed before each call.
+    Algorithmic bytes: both views' logits once (2 x B x K x V x 4) plus the
+    rejected row of both views once more per sequence (2 x B x V x 4).  Inputs
+    drawn on the device: AR logits N(0, 2), draft logits = AR + N(0, 1),
+    proposals = the draft's argmax, uniform draws."""
+    import torch
+    from lossless_diffusion_speculative_b200 import binding as ob
+    from lossless_diffusion_speculative_b200 import workloads as wl
+
+    w = wl.WORKLOADS[name]
+    B, K, V = w.B, w.K, w.vocab
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 * w.cid + 96)
+    ar = torch.randn((B, K, V), generator=g, device=dev) * 2.0
+    dr = ar + torch.randn((B, K, V), generator=g, device=dev)
+    prop = dr.argmax(dim=2).to(torch.int32).contiguous()
+    ua = torch.rand((B, K), generator=g, device=dev)
+    ur = torch.rand((B,), generator=g, device=dev)
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    nxt = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = torch.empty(ob.orthrus_rejection_workspace_size(B, K, V), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for it in range(3 + iters):
+            flush.zero_()
+            if it >= 3:
+                ev[it - 3][0].record()
+            ob.orthrus_rejection_verify(ar, dr, prop, ua, ur, 1.0, acc, nxt, ws, stream=stream)
+            if it >= 3:
+                ev[it - 3][1].record()
+        torch.cuda.synchronize()
+    us = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev])) * 1e3
+    nbytes = 2 * B * K * V * 4 + 2 * B * V * 4
+    gbs = nbytes / (us * 1e-6) / 1e9
+    out = {"workload": name, "B": B, "K": K, "V": V, "us_per_call": us, "bytes": nbytes,
+           "read_gbs": gbs, "frac_of_hbm": gbs / hbm, "mean_accepted": float(acc.float().mean()),
+           "iters": iters, "kernel": "rs_stats_kernel + rs_verify_kernel",
+           "timing": "median of CUDA events per call; L2 flushed before each call"}
+    del ar, dr, flush
     return out
 
 
@@ -547,9 +651,17 @@ def main():
                                                 hbm, CONFIG_ITERS,
                                                 st=st if name == w.name else None)
                 torch.cuda.empty_cache()
+            configs["qwen3_8b_step_fused_qkv"] = measure_fused_step(
+                "qwen3_8b_step", dev, stream, hbm, CONFIG_ITERS // 2,
+                st=st if w.name == "qwen3_8b_step" else None)
+            torch.cuda.empty_cache()
             for name in LM_HEAD_SET:
                 configs["lm_head_consensus_" + name] = measure_lm_head(name, dev, stream, hbm,
                                                                        CONFIG_ITERS)
+                torch.cuda.empty_cache()
+            for name in REJECT_SET:
+                configs["rejection_verify_" + name] = measure_rejection(name, dev, stream, hbm,
+                                                                        CONFIG_ITERS)
                 torch.cuda.empty_cache()
         torch.cuda.synchronize()
         clocks = sampler.stop()

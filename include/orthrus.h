@@ -363,6 +363,41 @@ ORTHRUS_API int orthrus_lm_head_consensus(const void *hidden, const void *lm_hea
                                           int32_t *argmax_out, void *workspace,
                                           size_t workspace_bytes, int32_t *status, void *stream);
 
+/*
+ * orthrus_qkv_project — one layer's QKV projection of a view's block, with the
+ * block's keys and values written straight into the cache rows that view's
+ * attention reads (section 2.3 "parallel projection": the diffusion head
+ * projects the anchor and K-1 masks in one forward pass; "structural
+ * verification": the filled block runs through the frozen AR head; section
+ * 2.1: both views attend over one shared KV cache).  It replaces the
+ * projection -> staging buffer -> orthrus_write_block round trip.
+ *
+ * For token row t = b * K + i (each fp32 sum rounded to bf16, nearest-even):
+ *     q_out[b, i, h, :]             = w_q[h*D : (h+1)*D, :] . x[b, i, :]
+ *     k_cache[b, g, ctx_b + i, :]   = w_k[g*D : (g+1)*D, :] . x[b, i, :]
+ *     v_cache[b, g, ctx_b + i, :]   = w_v[g*D : (g+1)*D, :] . x[b, i, :]
+ * with ctx_b = ctx_lens[b]; no other cache row is touched.
+ *
+ *   x            [B, K, hidden] bf16: the block's hidden states after the
+ *                layer's input norm.
+ *   w_q          [Hq * D, hidden] bf16; w_k, w_v [Hkv * D, hidden] bf16 (the
+ *                layer's projection weights, one row per output feature).
+ *   ctx_lens     [B] int32 (device).  A sequence with ctx_lens[b] < 0 or
+ *                ctx_lens[b] + K > S_max sets ORTHRUS_STATUS_CAPACITY and its
+ *                cache rows are not written.
+ *   q_out        [B, K, Hq, D] bf16 out.
+ *   k_cache, v_cache  [B, Hkv, S_max, D] bf16, rows [ctx_b, ctx_b + K) written.
+ * Model-specific steps between projection and attention that the pages do
+ * not describe (per-head RMSNorm of q and k, rotary embedding) are not applied.
+ * Supported: B * K <= ORTHRUS_MAX_LM_ROWS, hidden a multiple of 64, D a
+ * multiple of 16, Hq % Hkv == 0; x and the weights 16-byte aligned; sm_100
+ * devices only.  No workspace.
+ */
+ORTHRUS_API int orthrus_qkv_project(const void *x, const void *w_q, const void *w_k,
+                                    const void *w_v, const int32_t *ctx_lens, int B, int K,
+                                    int hidden, int Hq, int Hkv, int D, int S_max, void *q_out,
+                                    void *k_cache, void *v_cache, int32_t *status, void *stream);
+
 /* Human-readable text for an ORTHRUS_* return code (static storage). */
 ORTHRUS_API const char *orthrus_error_string(int code);
 

@@ -26,7 +26,7 @@ EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn", "orthrus_attn_path",
             "orthrus_kv_commit", "orthrus_write_block", "orthrus_error_string",
             "orthrus_version", "orthrus_lm_head_workspace_size",
             "orthrus_lm_head_consensus", "orthrus_rejection_workspace_size",
-            "orthrus_rejection_verify")
+            "orthrus_rejection_verify", "orthrus_qkv_project")
 
 
 class OrthrusError(RuntimeError):
@@ -75,6 +75,9 @@ def lib():
         L.orthrus_rejection_verify.restype = i32
         L.orthrus_rejection_verify.argtypes = [vp, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, vp, sz,
                                                vp, vp]
+        L.orthrus_qkv_project.restype = i32
+        L.orthrus_qkv_project.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp,
+                                          vp, vp, vp]
         L.orthrus_error_string.restype = ctypes.c_char_p
         L.orthrus_error_string.argtypes = [i32]
         L.orthrus_version.restype = i32
@@ -246,3 +249,22 @@ def orthrus_rejection_verify(ar_logits: torch.Tensor, draft_logits: torch.Tensor
                                         workspace.numel() * workspace.element_size(), _ptr(status),
                                         _stream(stream))
     _check("orthrus_rejection_verify", rc)
+
+
+def orthrus_qkv_project(x: torch.Tensor, w_q: torch.Tensor, w_k: torch.Tensor, w_v: torch.Tensor,
+                        ctx_lens: torch.Tensor, q_out: torch.Tensor, k_cache: torch.Tensor,
+                        v_cache: torch.Tensor, status: Optional[torch.Tensor] = None,
+                        stream=None) -> None:
+    """x [B,K,hidden] bf16, weights [features, hidden] bf16 -> q_out [B,K,Hq,D]
+    and cache rows [ctx, ctx+K) of k_cache / v_cache [B,Hkv,S_max,D] (bf16)."""
+    B, K, hidden = x.shape
+    _, Hkv, S_max, D = k_cache.shape
+    Hq = q_out.shape[2]
+    for t in (x, w_q, w_k, w_v, q_out, k_cache, v_cache):
+        assert t.dtype == torch.bfloat16
+    assert ctx_lens.dtype == torch.int32 and w_q.shape == (Hq * D, hidden)
+    assert w_k.shape == (Hkv * D, hidden) and w_v.shape == (Hkv * D, hidden)
+    rc = lib().orthrus_qkv_project(_ptr(x), _ptr(w_q), _ptr(w_k), _ptr(w_v), _ptr(ctx_lens), B, K,
+                                   hidden, Hq, Hkv, D, S_max, _ptr(q_out), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(status), _stream(stream))
+    _check("orthrus_qkv_project", rc)

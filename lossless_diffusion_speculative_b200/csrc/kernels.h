@@ -87,6 +87,19 @@ struct ConsensusArgs {
 };
 cudaError_t launch_consensus(const ConsensusArgs &p, cudaStream_t st);
 
+// Shape of one skinny-GEMM launch (skinny_gemm.cuh): weight rows in up to
+// three stacked segments against a few token rows.
+constexpr int kMaxSkinnySegs = 3;
+struct SkinnyShape {
+    int nseg;                            // weight segments (1..3)
+    int seg_end[kMaxSkinnySegs];         // segment s = rows [seg_end[s-1], seg_end[s])
+    int Hd;                              // hidden size (multiple of 64)
+    int BK;                              // token rows
+    int Np;                              // token rows padded for the MMA's N
+    int nst;                             // pipeline stages
+    int32_t *status;
+};
+
 // Fused AR LM head + argmax + consensus (lm_head.cu).
 constexpr int kMaxLmRows = ORTHRUS_MAX_LM_ROWS;   // B * K token rows per call
 struct LmHeadArgs {
@@ -96,11 +109,18 @@ struct LmHeadArgs {
     int32_t *argmax_out;
     unsigned long long *ws_keys;         // [B*K] packed (value, index) maxima, zero between calls
     unsigned int *ws_done;               // CTAs finished, zero between calls
-    int32_t *status;
-    int B, K, V, Hd;
-    int Np;                              // token rows padded for the MMA's N
-    int nst;                             // pipeline stages
-    int cps;                             // adjacent 64-wide hidden chunks per stage
+    int B, K, V;
+    SkinnyShape shape;
+};
+
+// The block's QKV projection written into the query buffer and the cache tail
+// (qkv_proj.cu).
+struct QkvArgs {
+    const int32_t *ctx_lens;
+    void *q_out;                         // [B, K, Hq, D] bf16
+    void *k_cache, *v_cache;             // [B, Hkv, S_max, D] bf16
+    int B, K, Hq, Hkv, D, S_max;
+    SkinnyShape shape;
 };
 
 // Rejection-sampling verification (rejection.cu).

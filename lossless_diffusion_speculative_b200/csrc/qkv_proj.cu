@@ -1,0 +1,192 @@
+// The block's QKV projection fused with the cache-tail write, for sm_100a.
+//
+// What it computes (Orthrus technical summary, gist.science, section 2.3:
+// "parallel projection" -- the diffusion head projects the anchor and K-1
+// masks in one forward pass -- and "structural verification" -- the filled
+// block runs through the frozen AR head; section 2.1: both views attend over
+// one shared KV cache): for one layer and one view, with x the block's hidden
+// states after the layer's input norm and token row t = b * K + i,
+//     q[b, i, h, :]               = W_q[h*D : (h+1)*D, :] x[t]
+//     k_cache[b, g, ctx_b + i, :] = W_k[g*D : (g+1)*D, :] x[t]
+//     v_cache[b, g, ctx_b + i, :] = W_v[g*D : (g+1)*D, :] x[t]
+// each fp32 sum rounded to bf16 (nearest, ties to even).  The view's block
+// keys and values land directly in the cache rows its attention reads,
+// [ctx_b, ctx_b + K): no staging buffer and no separate install copy.  The
+// model-specific elementwise steps between projection and attention (Qwen3's
+// per-head RMSNorm of q and k, rotary position embedding) are not on the pages
+// and not part of this call.
+//
+// The projections are the skinny GEMM of skinny_gemm.cuh over the stacked
+// weight rows [W_q; W_k; W_v] (three segments).  Epilogue: a warp's 32 lanes
+// hold 32 consecutive output features of one token row, so every bf16 store of
+// the warp is 64 contiguous bytes.  A sequence without room for its block
+// (ctx_b < 0 or ctx_b + K > S_max) is skipped and raises
+// ORTHRUS_STATUS_CAPACITY.
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "skinny_gemm.cuh"
+
+namespace orthrus {
+namespace qkv {
+
+using namespace sm100;
+
+template <int CPS>
+__global__ void __launch_bounds__(sg::kThreads, 1)
+    qkv_proj_kernel(const __grid_constant__ sg::Maps mp, const QkvArgs p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const sg::Shape &sp = p.shape;
+    sg::Smem sm;
+    pdl_trigger();
+    sg::prologue(sm, smem_raw, sp, CPS, 0, mp);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sg::tmem_base(sm);
+
+    // ---- everything below may read what earlier kernels wrote
+    pdl_wait();
+    const int cid = blockIdx.x, grid = gridDim.x;
+    if (cid == 0)
+        for (int b = threadIdx.x; b < p.B; b += sg::kThreads) {
+            const int c = p.ctx_lens[b];
+            if (c < 0 || (int64_t)c + p.K > p.S_max) raise_status(sp.status, ORTHRUS_STATUS_CAPACITY);
+        }
+    if (warp < 4) {
+        __nv_bfloat16 *q = static_cast<__nv_bfloat16 *>(p.q_out);
+        __nv_bfloat16 *kc = static_cast<__nv_bfloat16 *>(p.k_cache);
+        __nv_bfloat16 *vc = static_cast<__nv_bfloat16 *>(p.v_cache);
+        const int qrow = p.Hq * p.D;
+        sg::epilogue_tiles(sm, sp, cid, grid, tmem,
+                           [&](int row, int seg, int seg_lo, bool valid, int c0, const uint32_t (&x)[32]) {
+                               if (!valid) return;
+                               const int f = row - seg_lo;                   // feature in its segment
+                               const int g = f / p.D, d = f - g * p.D;       // (k, v: KV head, dim)
+                               __nv_bfloat16 *cache = seg == 1 ? kc : vc;
+#pragma unroll 4
+                               for (int c = 0; c < 32; ++c) {
+                                   const int t = c0 + c;
+                                   if (t >= sp.BK) break;
+                                   const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(x[c]));
+                                   if (seg == 0) {
+                                       q[(size_t)t * qrow + f] = v;
+                                   } else {
+                                       const int b = t / p.K, i = t - b * p.K;
+                                       const int ctx = __ldg(p.ctx_lens + b);
+                                       if (ctx < 0 || (int64_t)ctx + p.K > p.S_max) continue;
+                                       cache[(((size_t)b * p.Hkv + g) * p.S_max + ctx + i) * p.D + d] = v;
+                                   }
+                               }
+                           });
+    } else if (warp == 4) {
+        if (lane == 0) sg::producer<CPS>(sm, sp, mp, cid, grid);
+        __syncwarp();
+    } else {
+        if (lane == 0) sg::mma_issuer<CPS>(sm, sp, cid, grid, tmem);
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    sg::tmem_free(tmem);
+}
+
+}  // namespace qkv
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_qkv_once[kMaxDevices];
+bool g_qkv_ok[kMaxDevices];
+
+bool qkv_smem_ready(int dev)
+{
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::call_once(g_qkv_once[dev], [dev] {
+        const int lim = 227 * 1024;
+        g_qkv_ok[dev] =
+            cudaFuncSetAttribute(qkv::qkv_proj_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(qkv::qkv_proj_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(qkv::qkv_proj_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
+                cudaSuccess;
+        if (!g_qkv_ok[dev]) cudaGetLastError();
+    });
+    return g_qkv_ok[dev];
+}
+
+}  // namespace
+
+}  // namespace orthrus
+
+using namespace orthrus;
+
+extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w_k, const void *w_v,
+                                   const int32_t *ctx_lens, int B, int K, int hidden, int Hq, int Hkv,
+                                   int D, int S_max, void *q_out, void *k_cache, void *v_cache,
+                                   int32_t *status, void *stream)
+{
+    if (!x || !w_q || !w_k || !w_v || !ctx_lens || !q_out || !k_cache || !v_cache) return ORTHRUS_ERR_ARG;
+    if (B <= 0 || K <= 0 || hidden <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || K > S_max)
+        return ORTHRUS_ERR_ARG;
+    if ((int64_t)B * K > kMaxLmRows || hidden % 64 != 0 || D % 16 != 0 || Hq % Hkv != 0)
+        return ORTHRUS_ERR_UNSUPPORTED;
+    if ((int64_t)(Hq + 2 * Hkv) * D >= (1ll << 31) || (int64_t)B * Hkv * S_max * D >= (1ll << 40))
+        return ORTHRUS_ERR_UNSUPPORTED;
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)w_q | (uintptr_t)w_k | (uintptr_t)w_v;
+    if (al & 15u) return ORTHRUS_ERR_ALIGN;
+    int dev = 0, sms = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ERR_DEVICE;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (sms <= 0 || major != 10) return ORTHRUS_ERR_DEVICE;
+
+    QkvArgs a;
+    a.ctx_lens = ctx_lens;
+    a.q_out = q_out;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.B = B;
+    a.K = K;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    SkinnyShape &sp = a.shape;
+    sp.nseg = 3;
+    sp.seg_end[0] = Hq * D;
+    sp.seg_end[1] = sp.seg_end[0] + Hkv * D;
+    sp.seg_end[2] = sp.seg_end[1] + Hkv * D;
+    sp.Hd = hidden;
+    sp.BK = B * K;
+    sp.Np = sg::padded_n(B * K);
+    sp.status = status;
+    int cps = 1;
+    sg::pipeline_of(sp.Np, hidden / 64, &cps, &sp.nst);
+    const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, 0);
+
+    sg::Maps mp;
+    if (!sg::encode_w(mp, 0, w_q, Hq * D, hidden) || !sg::encode_w(mp, 1, w_k, Hkv * D, hidden) ||
+        !sg::encode_w(mp, 2, w_v, Hkv * D, hidden) || !sg::encode_x(mp, x, B * K, hidden, sp.Np))
+        return ORTHRUS_ERR_LAUNCH;
+    if (!qkv_smem_ready(dev)) return ORTHRUS_ERR_LAUNCH;
+    const int g16 = sp.seg_end[2] / 16;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g16 < sms ? g16 : sms);
+    cfg.blockDim = dim3(sg::kThreads);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cps == 4   ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<4>, mp, a)
+                          : cps == 2 ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<2>, mp, a)
+                                     : cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<1>, mp, a);
+    return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}

@@ -40,8 +40,8 @@ class StepResult:
 
 class DecodeStep:
     def __init__(self, w: wl.Workload, layers: Optional[int] = None, order: str = "cold",
-                 device: Optional[torch.device] = None):
-        assert order in ("cold", "interleaved")
+                 device: Optional[torch.device] = None, project: bool = False):
+        assert order in ("cold", "interleaved", "fused")
         self.w = w
         self.L = w.layers if layers is None else layers
         self.order = order
@@ -82,6 +82,29 @@ class DecodeStep:
                                    dtype=torch.uint8, device=dev)
         self.graphs = None
         self.tc_path = ob.orthrus_attn_path(B, Hq, Hkv, D, K, dt) == 1
+        self.project = False
+        if project:
+            self.enable_projection()
+
+    def enable_projection(self):
+        """The fused layer step: each view's block hidden states x and every
+        layer's projection weights (random, N(0, 1/hidden)), drawn on the device
+        from a seeded generator; orthrus_qkv_project writes q_all and the cache
+        tail, replacing the block install."""
+        if self.project:
+            return
+        w, dev, dt = self.w, self.dev, self.dtype
+        B, K, Hq, Hkv, D, Hd = w.B, w.K, w.Hq, w.Hkv, w.D, w.hidden
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 * w.cid + 95)
+        self.x_all = torch.randn((2, self.L, B, K, Hd), generator=g, device=dev).to(dt)
+        sc = 1.0 / Hd ** 0.5
+        self.w_qkv = []
+        for _ in range(self.L):
+            self.w_qkv.append(tuple(
+                (torch.randn((n * D, Hd), generator=g, device=dev) * sc).to(dt)
+                for n in (Hq, Hkv, Hkv)))
+        self.project = True
 
     # -- the hot path, as launch sequences ---------------------------------
     def _write_block(self, view, layers=None):
@@ -97,6 +120,20 @@ class DecodeStep:
     def _attn_view(self, view):
         for layer in range(self.L):
             self._attn(view, layer)
+
+    def _project(self, view, layer):
+        wq, wk, wv = self.w_qkv[layer]
+        ob.orthrus_qkv_project(self.x_all[view, layer], wq, wk, wv, self.ctx, self.q_all[view, layer],
+                               self.k_cache[layer], self.v_cache[layer], status=self.status)
+
+    def _fused_view(self, view):
+        for layer in range(self.L):
+            self._project(view, layer)
+            self._attn(view, layer)
+
+    def _project_view(self, view):
+        for layer in range(self.L):
+            self._project(view, layer)
 
     def _tail(self):
         w = self.w
@@ -114,6 +151,14 @@ class DecodeStep:
         start each group once its inputs have arrived.
         """
         order = self.order if order is None else order
+        if order == "fused":
+            # per layer: QKV projection (q + cache tail) -> attention, per view
+            return [("fused_diff", lambda: self._fused_view(ob.DIFF)),
+                    ("fused_ar", lambda: self._fused_view(ob.AR)),
+                    ("consensus_commit", self._tail)]
+        if order == "project_only":
+            return [("project_diff", lambda: self._project_view(ob.DIFF)),
+                    ("project_ar", lambda: self._project_view(ob.AR))]
         if order == "cold" and chunk > 0:
             segs = []
             for view, vn in ((ob.DIFF, "diff"), (ob.AR, "ar")):

@@ -293,3 +293,40 @@ def residual_cdf(ar_row: np.ndarray, draft_row: np.ndarray, temperature: float) 
     if r.sum() <= 0.0:
         r = p
     return np.cumsum(r)
+
+
+def qkv_project(x: np.ndarray, w_q: np.ndarray, w_k: np.ndarray, w_v: np.ndarray, D: int):
+    """float64 projections of a view's block ("Orthrus: Memory-Efficient
+    Parallel Token Generation via Dual-View Diffusion", gist.science technical
+    summary, section 2.3 "parallel projection" / "structural verification";
+    section 2.1: the block's keys and values join the one shared cache).
+
+    x [B, K, hidden]; w_q [Hq*D, hidden]; w_k, w_v [Hkv*D, hidden] (exact bf16
+    values in float32).  Returns q [B, K, Hq, D], k [B, K, Hkv, D], v [B, K,
+    Hkv, D] in float64 (one library matrix product each) and, for each output,
+    sum_d |x_d w_d|, the scale of a float32 accumulation's rounding error.
+    """
+    B, K, hidden = x.shape
+    xf = np.asarray(x, np.float64).reshape(B * K, hidden)
+    xa = np.abs(xf)
+    outs = []
+    for w in (w_q, w_k, w_v):
+        wf = np.asarray(w, np.float64)
+        H = wf.shape[0] // D
+        outs.append(((xf @ wf.T).reshape(B, K, H, D), (xa @ np.abs(wf).T).reshape(B, K, H, D)))
+    (q, qa), (k, ka), (v, va) = outs
+    return q, k, v, qa, ka, va
+
+
+def install_block_rows(k_cache: np.ndarray, v_cache: np.ndarray, k_blk: np.ndarray, v_blk: np.ndarray,
+                       ctx_lens: np.ndarray, S_max: int) -> None:
+    """Cache rows [ctx_b, ctx_b + K) of every KV head take the block's keys and
+    values (in place); a sequence without room (ctx_b < 0 or ctx_b + K > S_max)
+    is left untouched."""
+    B, K = k_blk.shape[:2]
+    for b in range(B):
+        c = int(ctx_lens[b])
+        if c < 0 or c + K > S_max:
+            continue
+        k_cache[b, :, c:c + K] = np.transpose(k_blk[b], (1, 0, 2))
+        v_cache[b, :, c:c + K] = np.transpose(v_blk[b], (1, 0, 2))

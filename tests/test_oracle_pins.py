@@ -518,3 +518,61 @@ def test_rejection_hand_cases():
         acc, nxt, _, cm = oracle.rejection_verify(ar2, dr2, np.array([[2]], np.int32), np.array([[0.9]]),
                                                   np.array([up]), 1.0)
         assert acc[0] == 0 and nxt[0] == n, (up, nxt)
+
+
+# --------------------------------------------------------------------------- QKV projection
+
+def test_qkv_project_bruteforce_tiny():
+    rng = np.random.default_rng(80)
+    B, K, hidden, Hq, Hkv, D = 2, 3, 16, 4, 2, 4
+    x = wl.round_to_bf16(rng.standard_normal((B, K, hidden), dtype=np.float32))
+    wq = wl.round_to_bf16(rng.standard_normal((Hq * D, hidden), dtype=np.float32))
+    wk = wl.round_to_bf16(rng.standard_normal((Hkv * D, hidden), dtype=np.float32))
+    wv = wl.round_to_bf16(rng.standard_normal((Hkv * D, hidden), dtype=np.float32))
+    q, k, v, qa, ka, va = oracle.qkv_project(x, wq, wk, wv, D)
+    for b in range(B):
+        for i in range(K):
+            for w, out, H in ((wq, q, Hq), (wk, k, Hkv), (wv, v, Hkv)):
+                for h in range(H):
+                    for d in range(D):
+                        row = w[h * D + d]
+                        exact = math.fsum(float(x[b, i, j]) * float(row[j]) for j in range(hidden))
+                        assert abs(out[b, i, h, d] - exact) < 1e-12
+    assert qa.shape == q.shape and (qa >= np.abs(q) - 1e-12).all()
+
+
+def test_qkv_project_feature_mapping_one_hot():
+    """One-hot weight rows: output feature h*D + d of a projection copies input
+    dimension (h*D + d) mod hidden, so the head and dim indices of q, k, v are
+    pinned to the weight rows."""
+    rng = np.random.default_rng(81)
+    B, K, hidden, Hq, Hkv, D = 2, 2, 40, 4, 2, 8
+    x = wl.round_to_bf16(rng.standard_normal((B, K, hidden), dtype=np.float32))
+    eye = lambda n: np.eye(hidden, dtype=np.float32)[np.arange(n) % hidden]
+    q, k, v, _, _, _ = oracle.qkv_project(x, eye(Hq * D), eye(Hkv * D) * 2, eye(Hkv * D) * 3, D)
+    for h in range(Hq):
+        for d in range(D):
+            assert (q[:, :, h, d] == x[:, :, (h * D + d) % hidden]).all()
+    for g in range(Hkv):
+        for d in range(D):
+            assert (k[:, :, g, d] == 2 * x[:, :, (g * D + d) % hidden]).all()
+            assert (v[:, :, g, d] == 3 * x[:, :, (g * D + d) % hidden]).all()
+
+
+def test_install_block_rows_places_the_tail_only():
+    rng = np.random.default_rng(82)
+    B, K, Hkv, D, S = 3, 4, 2, 5, 20
+    kc = rng.standard_normal((B, Hkv, S, D))
+    vc = rng.standard_normal((B, Hkv, S, D))
+    kb = rng.standard_normal((B, K, Hkv, D))
+    vb = rng.standard_normal((B, K, Hkv, D))
+    ctx = np.array([0, 9, S - K + 1], np.int32)            # the last has no room
+    k2, v2 = kc.copy(), vc.copy()
+    oracle.install_block_rows(k2, v2, kb, vb, ctx, S)
+    for b in range(2):
+        c = int(ctx[b])
+        for g in range(Hkv):
+            assert (k2[b, g, c:c + K] == kb[b, :, g]).all() and (v2[b, g, c:c + K] == vb[b, :, g]).all()
+            keep = np.r_[0:c, c + K:S]
+            assert (k2[b, g, keep] == kc[b, g, keep]).all() and (v2[b, g, keep] == vc[b, g, keep]).all()
+    assert (k2[2] == kc[2]).all() and (v2[2] == vc[2]).all()
