@@ -152,6 +152,40 @@ ORTHRUS_API int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void 
                  size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
+ * orthrus_prefill_workspace_size — scratch bytes for orthrus_prefill_attn
+ * (zero-fill once before first use, as for orthrus_attn).  0 for invalid sizes.
+ */
+ORTHRUS_API size_t orthrus_prefill_workspace_size(int B, int S, int Hq, int Hkv, int D,
+                                                  orthrus_dtype dtype);
+
+/*
+ * orthrus_prefill_attn — causal attention over a prompt whose keys and values
+ * already sit in the cache: the frozen AR head builds the shared cache's causal
+ * representation of the prompt (section 2.1), before any block is decoded.
+ *
+ *     out[b, s, h, :] = sum_{j <= s} softmax_j(scale * <q[b,s,h,:], k_cache[b,g,j,:]>) v_cache[b,g,j,:]
+ *
+ * for every sequence b, prompt position s < S and query head h (KV head
+ * g = h / (Hq/Hkv)).  It runs as chunked AR-view attention: prompt chunk c of
+ * Kc tokens is exactly an AR-view block after c * Kc context tokens, so the
+ * chunks of every sequence go to the tensor-core attention kernel as one
+ * batch reading their sequence's cache (Kc = the largest power of two with
+ * (Hq/Hkv) * Kc <= 128; a ragged tail of S mod Kc tokens is a second launch).
+ *
+ *   q        [B, S, Hq, D] (bf16 or fp32, as dtype).
+ *   k_cache, v_cache  [B, Hkv, S_max, D]; rows [0, S) hold the prompt's keys
+ *            and values.  S <= S_max.
+ *   out      [B, S, Hq, D] fp32.
+ *   workspace >= orthrus_prefill_workspace_size(B, S, Hq, Hkv, D, dtype)
+ *            bytes, 16-byte aligned, zero-filled once before first use.
+ * Supported shapes and alignment as orthrus_attn.
+ */
+ORTHRUS_API int orthrus_prefill_attn(orthrus_dtype dtype, const void *q, const void *k_cache,
+                                     const void *v_cache, int B, int S, int Hq, int Hkv, int D,
+                                     int S_max, float scale, float *out, void *workspace,
+                                     size_t workspace_bytes, int32_t *status, void *stream);
+
+/*
  * orthrus_consensus_workspace_size — scratch bytes for orthrus_consensus
  * (one packed (value, index) candidate per vocabulary chunk per row).
  */
@@ -389,14 +423,20 @@ ORTHRUS_API int orthrus_lm_head_consensus(const void *hidden, const void *lm_hea
  *   k_cache, v_cache  [B, Hkv, S_max, D] bf16, rows [ctx_b, ctx_b + K) written.
  * Model-specific steps between projection and attention that the pages do
  * not describe (per-head RMSNorm of q and k, rotary embedding) are not applied.
+ *   workspace    >= orthrus_qkv_workspace_size() bytes, 16-byte aligned,
+ *                zero-filled once before first use (its per-tile counters must
+ *                be zero when a call starts; every completed call leaves them
+ *                zero).  Calls that overlap on the device must not share it.
  * Supported: B * K <= ORTHRUS_MAX_LM_ROWS, hidden a multiple of 64, D a
- * multiple of 16, Hq % Hkv == 0; x and the weights 16-byte aligned; sm_100
- * devices only.  No workspace.
+ * multiple of 16, Hq % Hkv == 0; x, the weights and the workspace 16-byte
+ * aligned; sm_100 devices only.
  */
+ORTHRUS_API size_t orthrus_qkv_workspace_size(int B, int K, int hidden, int Hq, int Hkv, int D);
 ORTHRUS_API int orthrus_qkv_project(const void *x, const void *w_q, const void *w_k,
                                     const void *w_v, const int32_t *ctx_lens, int B, int K,
                                     int hidden, int Hq, int Hkv, int D, int S_max, void *q_out,
-                                    void *k_cache, void *v_cache, int32_t *status, void *stream);
+                                    void *k_cache, void *v_cache, void *workspace,
+                                    size_t workspace_bytes, int32_t *status, void *stream);
 
 /* Human-readable text for an ORTHRUS_* return code (static storage). */
 ORTHRUS_API const char *orthrus_error_string(int code);

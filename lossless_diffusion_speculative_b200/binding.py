@@ -26,7 +26,9 @@ EXPORTED = ("orthrus_attn_workspace_size", "orthrus_attn", "orthrus_attn_path",
             "orthrus_kv_commit", "orthrus_write_block", "orthrus_error_string",
             "orthrus_version", "orthrus_lm_head_workspace_size",
             "orthrus_lm_head_consensus", "orthrus_rejection_workspace_size",
-            "orthrus_rejection_verify", "orthrus_qkv_project")
+            "orthrus_rejection_verify", "orthrus_qkv_workspace_size", "orthrus_qkv_project",
+            "orthrus_prefill_workspace_size",
+            "orthrus_prefill_attn")
 
 
 class OrthrusError(RuntimeError):
@@ -75,9 +77,16 @@ def lib():
         L.orthrus_rejection_verify.restype = i32
         L.orthrus_rejection_verify.argtypes = [vp, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, vp, sz,
                                                vp, vp]
+        L.orthrus_qkv_workspace_size.restype = sz
+        L.orthrus_qkv_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.orthrus_qkv_project.restype = i32
         L.orthrus_qkv_project.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp,
-                                          vp, vp, vp]
+                                          vp, vp, sz, vp, vp]
+        L.orthrus_prefill_workspace_size.restype = sz
+        L.orthrus_prefill_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.orthrus_prefill_attn.restype = i32
+        L.orthrus_prefill_attn.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, sz,
+                                           vp, vp]
         L.orthrus_error_string.restype = ctypes.c_char_p
         L.orthrus_error_string.argtypes = [i32]
         L.orthrus_version.restype = i32
@@ -251,10 +260,14 @@ def orthrus_rejection_verify(ar_logits: torch.Tensor, draft_logits: torch.Tensor
     _check("orthrus_rejection_verify", rc)
 
 
+def orthrus_qkv_workspace_size(B: int, K: int, hidden: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().orthrus_qkv_workspace_size(B, K, hidden, Hq, Hkv, D))
+
+
 def orthrus_qkv_project(x: torch.Tensor, w_q: torch.Tensor, w_k: torch.Tensor, w_v: torch.Tensor,
                         ctx_lens: torch.Tensor, q_out: torch.Tensor, k_cache: torch.Tensor,
-                        v_cache: torch.Tensor, status: Optional[torch.Tensor] = None,
-                        stream=None) -> None:
+                        v_cache: torch.Tensor, workspace: torch.Tensor,
+                        status: Optional[torch.Tensor] = None, stream=None) -> None:
     """x [B,K,hidden] bf16, weights [features, hidden] bf16 -> q_out [B,K,Hq,D]
     and cache rows [ctx, ctx+K) of k_cache / v_cache [B,Hkv,S_max,D] (bf16)."""
     B, K, hidden = x.shape
@@ -266,5 +279,27 @@ def orthrus_qkv_project(x: torch.Tensor, w_q: torch.Tensor, w_k: torch.Tensor, w
     assert w_k.shape == (Hkv * D, hidden) and w_v.shape == (Hkv * D, hidden)
     rc = lib().orthrus_qkv_project(_ptr(x), _ptr(w_q), _ptr(w_k), _ptr(w_v), _ptr(ctx_lens), B, K,
                                    hidden, Hq, Hkv, D, S_max, _ptr(q_out), _ptr(k_cache),
-                                   _ptr(v_cache), _ptr(status), _stream(stream))
+                                   _ptr(v_cache), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _ptr(status),
+                                   _stream(stream))
     _check("orthrus_qkv_project", rc)
+
+
+def orthrus_prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, D: int,
+                                   dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib().orthrus_prefill_workspace_size(B, S, Hq, Hkv, D, _dtype_code(dtype)))
+
+
+def orthrus_prefill_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                         out: torch.Tensor, workspace: torch.Tensor, status: Optional[torch.Tensor] = None,
+                         scale: float = 0.0, stream=None) -> None:
+    """Causal attention over the prompt: q [B,S,Hq,D], caches [B,Hkv,S_max,D]
+    (rows [0, S) = the prompt) -> out [B,S,Hq,D] fp32."""
+    B, S, Hq, D = q.shape
+    _, Hkv, S_max, _ = k_cache.shape
+    assert out.dtype == torch.float32 and out.shape == q.shape
+    rc = lib().orthrus_prefill_attn(_dtype_code(q.dtype), _ptr(q), _ptr(k_cache), _ptr(v_cache), B, S, Hq,
+                                    Hkv, D, S_max, float(scale), _ptr(out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(status),
+                                    _stream(stream))
+    _check("orthrus_prefill_attn", rc)

@@ -99,10 +99,15 @@ size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K, orthrus
     return attn_ws_bytes(pl.slots, (Hq / Hkv) * K, D);
 }
 
-int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const void *k_cache,
-                 const void *v_cache, const int32_t *ctx_lens, int B, int Hq, int Hkv, int D,
-                 int S_max, int K, float scale, float *out, void *workspace,
-                 size_t workspace_bytes, int32_t *status, void *stream)
+}  // extern "C"
+
+namespace {
+
+// One attention launch (both paths).  cache_div / q_seq_rows: see AttnArgs.
+int attn_call(orthrus_view view, orthrus_dtype dtype, const void *q, const void *k_cache,
+              const void *v_cache, const int32_t *ctx_lens, int B, int Hq, int Hkv, int D, int S_max,
+              int K, float scale, float *out, void *workspace, size_t workspace_bytes, int32_t *status,
+              void *stream, int cache_div, int q_seq_rows)
 {
     if (view != ORTHRUS_DIFF && view != ORTHRUS_AR) return ORTHRUS_ERR_ARG;
     if (!q || !k_cache || !v_cache || !ctx_lens || !out) return ORTHRUS_ERR_ARG;
@@ -145,9 +150,103 @@ int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const vo
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
     a.scale_log2 = sc * kLog2e;
     a.min_keys = pl.min_keys;
+    a.cache_div = cache_div;
+    a.q_seq_rows = q_seq_rows;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const cudaError_t e = pl.tc ? launch_attn_tc(a, pl.grid, st) : launch_attn_simt(a, pl.grid, st);
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
+}
+
+// Chunked prefill: prompt chunk c of sequence s runs as call sequence
+// s * nch + c, an AR-view block of kc tokens after c * kc context tokens.
+__global__ void prefill_ctx_kernel(int32_t *ctx, int n, int nch, int kc, int offset)
+{
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < n) ctx[b] = (b % nch) * kc + offset;
+}
+
+int prefill_chunk(int G)
+{
+    int kc = 128;
+    while (kc > 1 && G * kc > 128) kc >>= 1;
+    return kc;
+}
+
+struct PrefillPlan {
+    int kc, nch, r;
+    size_t ws_attn, ctx_off, total;
+};
+
+PrefillPlan prefill_plan(int B, int S, int Hq, int Hkv, int D, orthrus_dtype dtype)
+{
+    PrefillPlan pp;
+    pp.kc = prefill_chunk(Hq / Hkv);
+    if (pp.kc > S) pp.kc = S;
+    pp.nch = S / pp.kc;
+    pp.r = S - pp.nch * pp.kc;
+    const size_t w1 = pp.nch ? orthrus_attn_workspace_size(B * pp.nch, Hq, Hkv, D, pp.kc, dtype) : 0;
+    const size_t w2 = pp.r ? orthrus_attn_workspace_size(B, Hq, Hkv, D, pp.r, dtype) : 0;
+    pp.ws_attn = ((w1 > w2 ? w1 : w2) + 255) & ~(size_t)255;
+    pp.ctx_off = pp.ws_attn;
+    pp.total = pp.ctx_off + (((size_t)B * (pp.nch + 1) * sizeof(int32_t) + 255) & ~(size_t)255);
+    if ((pp.nch && !w1) || (pp.r && !w2)) pp.total = 0;
+    return pp;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orthrus_attn(orthrus_view view, orthrus_dtype dtype, const void *q, const void *k_cache,
+                 const void *v_cache, const int32_t *ctx_lens, int B, int Hq, int Hkv, int D,
+                 int S_max, int K, float scale, float *out, void *workspace,
+                 size_t workspace_bytes, int32_t *status, void *stream)
+{
+    return attn_call(view, dtype, q, k_cache, v_cache, ctx_lens, B, Hq, Hkv, D, S_max, K, scale, out,
+                     workspace, workspace_bytes, status, stream, 1, K);
+}
+
+size_t orthrus_prefill_workspace_size(int B, int S, int Hq, int Hkv, int D, orthrus_dtype dtype)
+{
+    if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv) return 0;
+    return prefill_plan(B, S, Hq, Hkv, D, dtype).total;
+}
+
+int orthrus_prefill_attn(orthrus_dtype dtype, const void *q, const void *k_cache, const void *v_cache,
+                         int B, int S, int Hq, int Hkv, int D, int S_max, float scale, float *out,
+                         void *workspace, size_t workspace_bytes, int32_t *status, void *stream)
+{
+    if (!q || !k_cache || !v_cache || !out) return ORTHRUS_ERR_ARG;
+    if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || Hq % Hkv) return ORTHRUS_ERR_ARG;
+    if (S > S_max) return ORTHRUS_ERR_ARG;
+    if (dtype != ORTHRUS_BF16 && dtype != ORTHRUS_F32) return ORTHRUS_ERR_ARG;
+    const PrefillPlan pp = prefill_plan(B, S, Hq, Hkv, D, dtype);
+    if (!pp.total) return ORTHRUS_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < pp.total) return ORTHRUS_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ORTHRUS_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    int32_t *ctx1 = reinterpret_cast<int32_t *>(ws + pp.ctx_off);
+    int32_t *ctx2 = ctx1 + (size_t)B * pp.nch;
+    const size_t esz = dtype == ORTHRUS_BF16 ? 2 : 4;
+    if (pp.nch) {
+        const int n = B * pp.nch;
+        prefill_ctx_kernel<<<(n + 255) / 256, 256, 0, st>>>(ctx1, n, pp.nch, pp.kc, 0);
+        if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ERR_LAUNCH;
+        const int rc = attn_call(ORTHRUS_AR, dtype, q, k_cache, v_cache, ctx1, n, Hq, Hkv, D, S_max, pp.kc,
+                                 scale, out, ws, pp.ws_attn, status, stream, pp.nch, S);
+        if (rc != ORTHRUS_OK) return rc;
+    }
+    if (pp.r) {
+        prefill_ctx_kernel<<<(B + 255) / 256, 256, 0, st>>>(ctx2, B, 1, 0, pp.nch * pp.kc);
+        if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ERR_LAUNCH;
+        const size_t off = (size_t)pp.nch * pp.kc * Hq * D;
+        const int rc = attn_call(ORTHRUS_AR, dtype, static_cast<const char *>(q) + off * esz, k_cache, v_cache,
+                                 ctx2, B, Hq, Hkv, D, S_max, pp.r, scale, out + off, ws, pp.ws_attn, status,
+                                 stream, 1, S);
+        if (rc != ORTHRUS_OK) return rc;
+    }
+    return ORTHRUS_OK;
 }
 
 static void consensus_split(int B, int K, int V, int sms, int *splits, int *chunk)

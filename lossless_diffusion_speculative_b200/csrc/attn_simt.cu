@@ -39,12 +39,12 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs p)
         const int C = pc.len - p.K;
         const bool sole = (pc.a == 0 && pc.e == pc.len);
         const int slot = blockIdx.x + pc.s;
-        const T *kseg = kc + ((size_t)pc.b * p.Hkv + pc.g) * p.S_max * p.D;
-        const T *vseg = vc + ((size_t)pc.b * p.Hkv + pc.g) * p.S_max * p.D;
+        const T *kseg = kc + ((size_t)p.cache_seq(pc.b) * p.Hkv + pc.g) * p.S_max * p.D;
+        const T *vseg = vc + ((size_t)p.cache_seq(pc.b) * p.Hkv + pc.g) * p.S_max * p.D;
         for (int r = warp; r < rows; r += nwarps) {
             const int i = r / G;
             const int h = pc.g * G + (r % G);
-            const T *qr = q + (((size_t)pc.b * p.K + i) * p.Hq + h) * p.D;
+            const T *qr = q + ((p.q_row0(pc.b) + i) * p.Hq + h) * p.D;
             float qv[DPL], o[DPL];
 #pragma unroll
             for (int t = 0; t < DPL; ++t) {
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs p)
             }
             const float inv = l > 0.f ? 1.f / l : 0.f;
             if (sole) {
-                float *orow = p.out + (((size_t)pc.b * p.K + i) * p.Hq + h) * p.D;
+                float *orow = p.out + ((p.q_row0(pc.b) + i) * p.Hq + h) * p.D;
 #pragma unroll
                 for (int t = 0; t < DPL; ++t) orow[lane + 32 * t] = o[t] * inv;
             } else {
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) attn_combine_kernel(AttnAr
     const float inv = 1.f / wsum;
     const int i = r / G;
     const int h = g * G + (r % G);
-    float4 *orow = reinterpret_cast<float4 *>(p.out + (((size_t)b * p.K + i) * p.Hq + h) * p.D);
+    float4 *orow = reinterpret_cast<float4 *>(p.out + ((p.q_row0(b) + i) * p.Hq + h) * p.D);
     const float4 *src = reinterpret_cast<const float4 *>(p.ws_o + ((size_t)(c_lo + s) * rows + r) * p.D);
     const size_t stride4 = (size_t)rows * p.D / 4;          // one split further
     for (int d4 = lane; d4 < p.D / 4; d4 += 32) {

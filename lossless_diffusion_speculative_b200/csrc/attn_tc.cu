@@ -371,6 +371,7 @@ struct Tiling {
 struct SplitInfo {
     int b, g, s, c_lo, n;
     bool hi_last;
+    size_t row0;     // the sequence's first query / output row
 };
 // What the epilogue records of a shared piece (in shared memory, so that
 // nothing stays live in registers across the tile loop).
@@ -417,15 +418,16 @@ __device__ __forceinline__ void producer(const Shared &sh, const AttnArgs &p, co
             break;
         }
         mbar_expect_tx(sh.bar(B_QFULL), q_bytes);
-        tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, pc.b * p.K);
-        tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, pc.b * p.K);
+        const int qy = (int)p.q_row0(pc.b);
+        tma_load_3d(sh.base + kSmemQ, tq, sh.bar(B_QFULL), 0, pc.g * G, qy);
+        tma_load_3d(sh.base + kSmemQ + kHalfBytes, tq, sh.bar(B_QFULL), 64, pc.g * G, qy);
         ++qloads;
         // the K and V rings held the previous piece's output rows
         if (piece > 0 && !wait_bar(sh.bar(B_MERGED), (piece - 1) & 1, sh.abort_flag, p.status)) {
             ok = false;
             break;
         }
-        const int z = pc.b * p.Hkv + pc.g;
+        const int z = p.cache_seq(pc.b) * p.Hkv + pc.g;
         int nk = 0, nv = 0;                      // this piece's K and V tiles issued
         unsigned long long t0 = 0;
         uint32_t idle = 0;
@@ -763,11 +765,11 @@ __device__ __noinline__ int split_merge(uint32_t base, volatile int *abort_flag,
         }
         __syncwarp();                                         // wsm is rewritten next
         int row = r_lo + r;
-        float *dst = out + (((size_t)sp.b * K + row / G) * Hq + sp.g * G + row % G) * kD;
+        float *dst = out + ((sp.row0 + row / G) * Hq + sp.g * G + row % G) * kD;
         reinterpret_cast<float4 *>(dst)[lane] = make_float4(a0.x * inv0, a0.y * inv0, a1.x * inv0, a1.y * inv0);
         if (r1 != r) {
             row = r_lo + r1;
-            dst = out + (((size_t)sp.b * K + row / G) * Hq + sp.g * G + row % G) * kD;
+            dst = out + ((sp.row0 + row / G) * Hq + sp.g * G + row % G) * kD;
             reinterpret_cast<float4 *>(dst)[lane] = make_float4(b0.x * inv1, b0.y * inv1, b1.x * inv1, b1.y * inv1);
         }
     }
@@ -943,7 +945,7 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
                 stage_row(reinterpret_cast<float4 *>(smem + kSmemStage) + m * (kStagePitch / 4), 0);
                 fence_proxy_async();              // the row is visible to the bulk copy
                 if (row_ok) {
-                    bulk_store(p.out + (((size_t)pc.b * p.K + i) * p.Hq + pc.g * G + m % G) * kD,
+                    bulk_store(p.out + ((p.q_row0(pc.b) + i) * p.Hq + pc.g * G + m % G) * kD,
                                sh.base + kSmemStage + m * kStagePitch * 4, kD * 4);
                     bulk_commit();
                 }
@@ -999,6 +1001,7 @@ __device__ __forceinline__ bool softmax_epilogue(const Shared &sh, uint8_t *smem
         const int c_hi = plan_cta_of(plan, sp.s0 + sp.nbx - 1);
         si.n = c_hi - si.c_lo + 1;
         si.hi_last = plan_start(plan, c_hi + 1) <= sp.s0 + sp.nbx;
+        si.row0 = p.q_row0(sp.b);
         return si;
     };
     for (int k = 0; k < npend; ++k) {
@@ -1184,11 +1187,11 @@ cudaError_t launch_attn_tc(const AttnArgs &p, int units, cudaStream_t st)
     const int G = p.Hq / p.Hkv;
     CUtensorMap tq, tk, tv;
     const uint64_t row = tc::kD * 2;
-    if (!encode_3d(&tq, p.q, tc::kD, p.Hq, (uint64_t)p.B * p.K, row, (uint64_t)p.Hq * row, 64, G, p.K) ||
-        !encode_3d(&tk, p.k_cache, tc::kD, p.S_max, (uint64_t)p.B * p.Hkv, row,
-                   (uint64_t)p.S_max * row, 64, 64, 1) ||
-        !encode_3d(&tv, p.v_cache, tc::kD, p.S_max, (uint64_t)p.B * p.Hkv, row,
-                   (uint64_t)p.S_max * row, 64, 64, 1))
+    const uint64_t q_rows = (uint64_t)((p.B + p.cache_div - 1) / p.cache_div) * p.q_seq_rows;
+    const uint64_t kv_seqs = (uint64_t)((p.B + p.cache_div - 1) / p.cache_div) * p.Hkv;
+    if (!encode_3d(&tq, p.q, tc::kD, p.Hq, q_rows, row, (uint64_t)p.Hq * row, 64, G, p.K) ||
+        !encode_3d(&tk, p.k_cache, tc::kD, p.S_max, kv_seqs, row, (uint64_t)p.S_max * row, 64, 64, 1) ||
+        !encode_3d(&tv, p.v_cache, tc::kD, p.S_max, kv_seqs, row, (uint64_t)p.S_max * row, 64, 64, 1))
         return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(units);

@@ -26,6 +26,18 @@ struct AttnArgs {
     int dtype;           // orthrus_dtype
     float scale_log2;    // softmax scale * log2(e)
     int min_keys;        // smallest key range worth a CTA
+    // Sequence b of the call reads the cache of sequence b / cache_div and the
+    // query / output rows from q_row0(b); a decode call has cache_div = 1 and
+    // q_seq_rows = K (rows b * K).  Chunked prefill runs prompt chunk c of
+    // sequence s as call sequence s * cache_div + c.
+    int cache_div;
+    int q_seq_rows;
+    __host__ __device__ __forceinline__ int cache_seq(int b) const { return cache_div == 1 ? b : b / cache_div; }
+    __host__ __device__ __forceinline__ size_t q_row0(int b) const
+    {
+        return cache_div == 1 ? (size_t)b * q_seq_rows
+                              : (size_t)(b / cache_div) * q_seq_rows + (size_t)(b % cache_div) * K;
+    }
 };
 
 // Workspace layout shared by the attention paths: a fixed block of flags and
@@ -98,6 +110,12 @@ struct SkinnyShape {
     int Np;                              // token rows padded for the MMA's N
     int nst;                             // pipeline stages
     int32_t *status;
+    // split-K (ksplit > 1): CTA u computes tile u / ksplit over hidden chunks
+    // [k0(u % ksplit), k0(u % ksplit + 1)) into an fp32 partial; the last
+    // split of a tile (per-tile counter) sums the partials in split order
+    int ksplit;
+    float *ws_part;                      // [ksplit, rows, Np rounded up to 32] fp32 partials
+    unsigned int *ws_count;              // [tiles] splits done, zero between calls
 };
 
 // Fused AR LM head + argmax + consensus (lm_head.cu).

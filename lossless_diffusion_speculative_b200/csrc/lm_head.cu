@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     pdl_wait();
     const int cid = blockIdx.x, grid = gridDim.x;
     if (warp < 4) {
-        sg::epilogue_tiles(sm, sp, cid, grid, tmem,
+        sg::epilogue_tiles<false>(sm, sp, cid, grid, tmem, CPS,
                            [&](int row, int, int, bool valid, int c0, const uint32_t (&x)[32]) {
                                uint64_t k[32];
 #pragma unroll
@@ -172,7 +172,7 @@ bool lm_smem_ready(int dev)
 {
     if (dev < 0 || dev >= kMaxDevices) return false;
     std::call_once(g_smem_once[dev], [dev] {
-        const int lim = 227 * 1024;
+        const int lim = 226 * 1024;            // (room for the kernels' few bytes of static shared memory)
         g_smem_ok[dev] =
             cudaFuncSetAttribute(lmh::lm_head_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
                 cudaSuccess &&
@@ -236,6 +236,9 @@ int orthrus_lm_head_consensus(const void *hidden, const void *lm_head, const int
     sp.BK = BK;
     sp.Np = sg::padded_n(BK);
     sp.status = status;
+    sp.ksplit = 1;
+    sp.ws_part = nullptr;
+    sp.ws_count = nullptr;
     int cps = 1;
     sg::pipeline_of(sp.Np, Hd / 64, &cps, &sp.nst);
     const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, lmh::kExtraBytes);

@@ -17,7 +17,9 @@
 // and not part of this call.
 //
 // The projections are the skinny GEMM of skinny_gemm.cuh over the stacked
-// weight rows [W_q; W_k; W_v] (three segments).  Epilogue: a warp's 32 lanes
+// weight rows [W_q; W_k; W_v] (three segments); with fewer 128-row tiles than
+// half the SMs (Qwen3-8B: 48 tiles) the hidden dimension is split over
+// several CTAs per tile and the last split sums the fp32 partials.  Epilogue: a warp's 32 lanes
 // hold 32 consecutive output features of one token row, so every bf16 store of
 // the warp is 64 contiguous bytes.  A sequence without room for its block
 // (ctx_b < 0 or ctx_b + K > S_max) is skipped and raises
@@ -33,7 +35,7 @@ namespace qkv {
 
 using namespace sm100;
 
-template <int CPS>
+template <int CPS, bool SPLITK>
 __global__ void __launch_bounds__(sg::kThreads, 1)
     qkv_proj_kernel(const __grid_constant__ sg::Maps mp, const QkvArgs p)
 {
@@ -60,25 +62,27 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
         __nv_bfloat16 *q = static_cast<__nv_bfloat16 *>(p.q_out);
         __nv_bfloat16 *kc = static_cast<__nv_bfloat16 *>(p.k_cache);
         __nv_bfloat16 *vc = static_cast<__nv_bfloat16 *>(p.v_cache);
-        const int qrow = p.Hq * p.D;
-        sg::epilogue_tiles(sm, sp, cid, grid, tmem,
-                           [&](int row, int seg, int seg_lo, bool valid, int c0, const uint32_t (&x)[32]) {
+        const int qrow = p.Hq * p.D, D = p.D, K = p.K, Hkv = p.Hkv, S_max = p.S_max, BK = sp.BK;
+        const int32_t *ctx_lens = p.ctx_lens;
+        sg::epilogue_tiles<SPLITK>(sm, sp, cid, grid, tmem, CPS,
+                           [=](int row, int seg, int seg_lo, bool valid, int c0, const uint32_t (&x)[32]) {
                                if (!valid) return;
                                const int f = row - seg_lo;                   // feature in its segment
-                               const int g = f / p.D, d = f - g * p.D;       // (k, v: KV head, dim)
+                               const int g = f / D, d = f - g * D;           // (k, v: KV head, dim)
                                __nv_bfloat16 *cache = seg == 1 ? kc : vc;
-#pragma unroll 4
+#pragma unroll
                                for (int c = 0; c < 32; ++c) {
                                    const int t = c0 + c;
-                                   if (t >= sp.BK) break;
-                                   const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(x[c]));
-                                   if (seg == 0) {
-                                       q[(size_t)t * qrow + f] = v;
-                                   } else {
-                                       const int b = t / p.K, i = t - b * p.K;
-                                       const int ctx = __ldg(p.ctx_lens + b);
-                                       if (ctx < 0 || (int64_t)ctx + p.K > p.S_max) continue;
-                                       cache[(((size_t)b * p.Hkv + g) * p.S_max + ctx + i) * p.D + d] = v;
+                                   if (t < BK) {
+                                       const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(x[c]));
+                                       if (seg == 0) {
+                                           q[(size_t)t * qrow + f] = v;
+                                       } else {
+                                           const int b = t / K, i = t - b * K;
+                                           const int ctx = __ldg(ctx_lens + b);
+                                           if (ctx >= 0 && (int64_t)ctx + K <= S_max)
+                                               cache[(((size_t)b * Hkv + g) * S_max + ctx + i) * D + d] = v;
+                                       }
                                    }
                                }
                            });
@@ -106,14 +110,14 @@ bool qkv_smem_ready(int dev)
 {
     if (dev < 0 || dev >= kMaxDevices) return false;
     std::call_once(g_qkv_once[dev], [dev] {
-        const int lim = 227 * 1024;
-        g_qkv_ok[dev] =
-            cudaFuncSetAttribute(qkv::qkv_proj_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess &&
-            cudaFuncSetAttribute(qkv::qkv_proj_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess &&
-            cudaFuncSetAttribute(qkv::qkv_proj_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess;
+        const int lim = 226 * 1024;            // (room for the kernels' few bytes of static shared memory)
+        const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        g_qkv_ok[dev] = cudaFuncSetAttribute(qkv::qkv_proj_kernel<1, false>, at, lim) == cudaSuccess &&
+                        cudaFuncSetAttribute(qkv::qkv_proj_kernel<2, false>, at, lim) == cudaSuccess &&
+                        cudaFuncSetAttribute(qkv::qkv_proj_kernel<4, false>, at, lim) == cudaSuccess &&
+                        cudaFuncSetAttribute(qkv::qkv_proj_kernel<1, true>, at, lim) == cudaSuccess &&
+                        cudaFuncSetAttribute(qkv::qkv_proj_kernel<2, true>, at, lim) == cudaSuccess &&
+                        cudaFuncSetAttribute(qkv::qkv_proj_kernel<4, true>, at, lim) == cudaSuccess;
         if (!g_qkv_ok[dev]) cudaGetLastError();
     });
     return g_qkv_ok[dev];
@@ -125,10 +129,60 @@ bool qkv_smem_ready(int dev)
 
 using namespace orthrus;
 
+namespace {
+
+// Split-K plan: with fewer 128-row tiles than half the SMs, every tile's
+// hidden dimension is split over ksplit CTAs (one unit each).
+struct QkvPlan {
+    int Np, cps, nst, ntiles, ksplit, grid;
+    size_t part_bytes, total;
+};
+
+QkvPlan qkv_plan(int B, int K, int hidden, int Hq, int Hkv, int D, int sms)
+{
+    QkvPlan q;
+    q.Np = sg::padded_n(B * K);
+    sg::pipeline_of(q.Np, hidden / 64, &q.cps, &q.nst);
+    const int rows[3] = {Hq * D, Hkv * D, Hkv * D};
+    q.ntiles = 0;
+    for (int r : rows) q.ntiles += (r + sg::kTileRows - 1) / sg::kTileRows;
+    const int units = hidden / 64 / q.cps;
+    q.ksplit = 1;
+    if (2 * q.ntiles <= sms) {
+        q.ksplit = sms / q.ntiles;
+        if (q.ksplit > units) q.ksplit = units;
+    }
+    const int g16 = (Hq + 2 * Hkv) * D / 16;
+    q.grid = q.ksplit > 1 ? q.ntiles * q.ksplit : (g16 < sms ? g16 : sms);
+    const size_t ldp = (size_t)((q.Np + 31) & ~31);         // partial row stride (floats)
+    q.part_bytes = q.ksplit > 1 ? (((size_t)q.ksplit * (Hq + 2 * Hkv) * D * ldp * 4 + 255) & ~(size_t)255) : 0;
+    q.total = q.part_bytes + (((size_t)q.ntiles * 4 + 255) & ~(size_t)255);
+    return q;
+}
+
+int qkv_sms()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+}  // namespace
+
+extern "C" size_t orthrus_qkv_workspace_size(int B, int K, int hidden, int Hq, int Hkv, int D)
+{
+    if (B <= 0 || K <= 0 || hidden <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || hidden % 64 != 0) return 0;
+    if ((int64_t)B * K > kMaxLmRows) return 0;
+    const int sms = qkv_sms();
+    if (sms <= 0) return 0;
+    return qkv_plan(B, K, hidden, Hq, Hkv, D, sms).total;
+}
+
 extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w_k, const void *w_v,
                                    const int32_t *ctx_lens, int B, int K, int hidden, int Hq, int Hkv,
                                    int D, int S_max, void *q_out, void *k_cache, void *v_cache,
-                                   int32_t *status, void *stream)
+                                   void *workspace, size_t workspace_bytes, int32_t *status, void *stream)
 {
     if (!x || !w_q || !w_k || !w_v || !ctx_lens || !q_out || !k_cache || !v_cache) return ORTHRUS_ERR_ARG;
     if (B <= 0 || K <= 0 || hidden <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S_max <= 0 || K > S_max)
@@ -137,7 +191,7 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
         return ORTHRUS_ERR_UNSUPPORTED;
     if ((int64_t)(Hq + 2 * Hkv) * D >= (1ll << 31) || (int64_t)B * Hkv * S_max * D >= (1ll << 40))
         return ORTHRUS_ERR_UNSUPPORTED;
-    const uintptr_t al = (uintptr_t)x | (uintptr_t)w_q | (uintptr_t)w_k | (uintptr_t)w_v;
+    const uintptr_t al = (uintptr_t)x | (uintptr_t)w_q | (uintptr_t)w_k | (uintptr_t)w_v | (uintptr_t)workspace;
     if (al & 15u) return ORTHRUS_ERR_ALIGN;
     int dev = 0, sms = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ERR_DEVICE;
@@ -156,6 +210,8 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
     a.Hkv = Hkv;
     a.D = D;
     a.S_max = S_max;
+    const QkvPlan qp = qkv_plan(B, K, hidden, Hq, Hkv, D, sms);
+    if (!workspace || workspace_bytes < qp.total) return ORTHRUS_ERR_WORKSPACE;
     SkinnyShape &sp = a.shape;
     sp.nseg = 3;
     sp.seg_end[0] = Hq * D;
@@ -163,10 +219,13 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
     sp.seg_end[2] = sp.seg_end[1] + Hkv * D;
     sp.Hd = hidden;
     sp.BK = B * K;
-    sp.Np = sg::padded_n(B * K);
+    sp.Np = qp.Np;
+    sp.nst = qp.nst;
     sp.status = status;
-    int cps = 1;
-    sg::pipeline_of(sp.Np, hidden / 64, &cps, &sp.nst);
+    sp.ksplit = qp.ksplit;
+    sp.ws_part = static_cast<float *>(workspace);
+    sp.ws_count = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + qp.part_bytes);
+    const int cps = qp.cps;
     const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, 0);
 
     sg::Maps mp;
@@ -174,9 +233,8 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
         !sg::encode_w(mp, 2, w_v, Hkv * D, hidden) || !sg::encode_x(mp, x, B * K, hidden, sp.Np))
         return ORTHRUS_ERR_LAUNCH;
     if (!qkv_smem_ready(dev)) return ORTHRUS_ERR_LAUNCH;
-    const int g16 = sp.seg_end[2] / 16;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(g16 < sms ? g16 : sms);
+    cfg.gridDim = dim3(qp.grid);
     cfg.blockDim = dim3(sg::kThreads);
     cfg.dynamicSmemBytes = L.total;
     cfg.stream = static_cast<cudaStream_t>(stream);
@@ -185,8 +243,16 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cps == 4   ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<4>, mp, a)
-                          : cps == 2 ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<2>, mp, a)
-                                     : cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<1>, mp, a);
+    const bool sk = qp.ksplit > 1;
+    cudaError_t e;
+    if (cps == 4)
+        e = sk ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<4, true>, mp, a)
+               : cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<4, false>, mp, a);
+    else if (cps == 2)
+        e = sk ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<2, true>, mp, a)
+               : cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<2, false>, mp, a);
+    else
+        e = sk ? cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<1, true>, mp, a)
+               : cudaLaunchKernelEx(&cfg, qkv::qkv_proj_kernel<1, false>, mp, a);
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }

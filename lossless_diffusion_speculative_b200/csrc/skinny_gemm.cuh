@@ -55,6 +55,7 @@ enum : int {
 
 using Shape = SkinnyShape;
 static_assert(kMaxSkinnySegs == kMaxSegs, "segments");
+static_assert(kRingBudget + (B_COUNT * 8 + 32) + 2 * 1024 * 8 + 1024 <= 226 * 1024, "layouts fit the 226 KiB limit");
 
 struct Maps {                            // one launch's tensor maps
     CUtensorMap w[kMaxSegs];             // box (64, 128) per weight segment
@@ -91,21 +92,48 @@ struct Smem {
     __device__ __forceinline__ uint8_t *extra() const { return ptr + L.extra; }
 };
 
-// The tiles of CTA `cid`'s range, in order; identical in every role.
+// Hidden-chunk range of split s of ksplit over nk chunks (multiples of cps).
+__host__ __device__ __forceinline__ int split_k0(int s, int ksplit, int nk, int cps)
+{
+    const int units = nk / cps;
+    return cps * (s * units / ksplit);
+}
+
+// The tiles of CTA `cid`'s range, in order; identical in every role.  Without
+// split-K the rows are cut into 16-row granules over the grid; with split-K
+// CTA cid owns 128-row tile cid / ksplit (tiles counted per segment) and the
+// hidden chunks [k_lo, k_hi) of split cid % ksplit.
 struct TileIter {
     int r0, hi;
     int e0, e1, e2;                      // segment ends (unused segments end at the last)
-    __device__ __forceinline__ TileIter(const Shape &sh, int cid, int grid)
+    int k_lo, k_hi;                      // hidden chunks of every tile
+    __device__ __forceinline__ TileIter(const Shape &sh, int cid, int grid, int cps)
     {
         e0 = sh.seg_end[0];
         e1 = sh.nseg > 1 ? sh.seg_end[1] : e0;
         e2 = sh.nseg > 2 ? sh.seg_end[2] : e1;
+        const int nk = sh.Hd / kChunk;
+        if (sh.ksplit > 1) {
+            int t = cid / sh.ksplit;
+            const int s = cid - (cid / sh.ksplit) * sh.ksplit;
+            const int n0 = (e0 + kTileRows - 1) / kTileRows;
+            const int n1 = (e1 - e0 + kTileRows - 1) / kTileRows;
+            r0 = t < n0 ? t * kTileRows : t < n0 + n1 ? e0 + (t - n0) * kTileRows : e1 + (t - n0 - n1) * kTileRows;
+            const int seg_hi = t < n0 ? e0 : t < n0 + n1 ? e1 : e2;
+            hi = r0 + kTileRows < seg_hi ? r0 + kTileRows : seg_hi;
+            if (r0 >= e2) r0 = hi = e2;
+            k_lo = split_k0(s, sh.ksplit, nk, cps);
+            k_hi = split_k0(s + 1, sh.ksplit, nk, cps);
+            return;
+        }
         const int rows = e2;
         const int g16 = (rows + 15) >> 4;
         const int q = g16 / grid, r = g16 - q * grid;
         r0 = 16 * (cid * q + (cid * r) / grid);
         hi = 16 * ((cid + 1) * q + ((cid + 1) * r) / grid);
         if (hi > rows) hi = rows;
+        k_lo = 0;
+        k_hi = nk;
     }
     // next tile [a, b) of weight segment `seg` (segment-local rows a - seg_lo)
     __device__ __forceinline__ bool next(int &a, int &b, int &seg, int &seg_lo)
@@ -129,15 +157,16 @@ __device__ __forceinline__ void producer(const Smem &sm, const Shape &sp, const 
     const int nk = sp.Hd / kChunk;
     const int half = sp.Np > 256 ? sp.Np / 2 : sp.Np;
     const uint64_t pol_w = make_policy_evict_first(), pol_x = make_policy_evict_last();
-    TileIter ti(sp, cid, grid);
+    TileIter ti(sp, cid, grid, CPS);
     int a, b, seg, seg_lo;
     uint32_t it = 0;
     bool ok = true;
+    (void)nk;
     while (ok && ti.next(a, b, seg, seg_lo)) {
         const int nrows = b - a, y0 = a - seg_lo;
         const int nb16 = (nrows + 15) >> 4;
         const uint32_t a_bytes = nrows == kTileRows ? kABytes : (uint32_t)nb16 * 16u * 128u;
-        for (int ks = 0; ks < nk / CPS; ++ks, ++it) {
+        for (int ks = ti.k_lo / CPS; ks < ti.k_hi / CPS; ++ks, ++it) {
             const int st = it % sp.nst;
             const uint32_t n = it / sp.nst;
             if (n > 0 && !wait_bar(sm.bar(B_EMPTY + st), (n - 1) & 1, sm.abort_flag, sp.status)) {
@@ -179,10 +208,11 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
     const bool split = sp.Np > 256;
     const int n_mma = split ? sp.Np / 2 : sp.Np;
     const uint32_t idesc = instr_desc(128, n_mma, false);
-    TileIter ti(sp, cid, grid);
+    TileIter ti(sp, cid, grid, CPS);
     int a, b, seg, seg_lo;
     uint32_t it = 0;
     bool ok = true;
+    (void)nk;
     for (int t = 0; ok && ti.next(a, b, seg, seg_lo); ++t) {
         const int acc = t % nacc;
         if (t >= nacc && !wait_bar(sm.bar(B_AEMPTY + acc), (t / nacc - 1) & 1, sm.abort_flag, sp.status)) {
@@ -191,7 +221,8 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
         }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * sp.Np);
-        for (int ks = 0; ks < nk / CPS; ++ks, ++it) {
+        const int ks0 = ti.k_lo / CPS;
+        for (int ks = ks0; ks < ti.k_hi / CPS; ++ks, ++it) {
             const int st = it % sp.nst;
             if (!wait_bar(sm.bar(B_FULL + st), (it / sp.nst) & 1, sm.abort_flag, sp.status)) {
                 ok = false;
@@ -206,7 +237,7 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
                 const uint64_t bd2 = smem_desc(xb + (uint32_t)n_mma * 128u, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {        // 16 hidden dims (32 bytes) per MMA
-                    const uint32_t on = (ks | j | kk) ? 1u : 0u;
+                    const uint32_t on = ((ks - ks0) | j | kk) ? 1u : 0u;
                     tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, on);
                     if (split) tc_mma_ss(d + (uint32_t)n_mma, ad + 2 * kk, bd2 + 2 * kk, idesc, on);
                 }
@@ -225,14 +256,18 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
 // f(row, seg, seg_lo, valid, col0, x) where row is this thread's weight row,
 // valid says it lies in the tile, and x[c] holds D[row, col0 + c] (fp32 bits).
 // Returns false after an abort.
-template <class F>
+// With split-K each split writes its fp32 partial; the last split of the
+// tile to finish (per-tile counter, acquire/release) sums the partials in
+// split order and calls f with the sums.  named barrier 1 joins warps 0-3.
+template <bool SPLITK, class F>
 __device__ __forceinline__ bool epilogue_tiles(const Smem &sm, const Shape &sp, int cid, int grid, uint32_t tmem,
-                                               F &&f)
+                                               int cps, F &&f)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nacc = 2 * sp.Np <= kTmemCols ? 2 : 1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    TileIter ti(sp, cid, grid);
+    const int rows = sp.seg_end[sp.nseg - 1];
+    TileIter ti(sp, cid, grid, cps);
     int a, b, seg, seg_lo;
     for (int t = 0; ti.next(a, b, seg, seg_lo); ++t) {
         const int acc = t % nacc;
@@ -240,11 +275,61 @@ __device__ __forceinline__ bool epilogue_tiles(const Smem &sm, const Shape &sp, 
         tc_fence_after();
         const int row = a + warp * 32 + lane;
         const bool valid = row < b;
-        for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
-            uint32_t x[32];
-            tmem_ld32(lane_base + (uint32_t)(acc * sp.Np + c0), x);
-            tmem_wait_ld();
-            f(row, seg, seg_lo, valid, c0, x);
+        if constexpr (!SPLITK) {
+            for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
+                uint32_t x[32];
+                tmem_ld32(lane_base + (uint32_t)(acc * sp.Np + c0), x);
+                tmem_wait_ld();
+                f(row, seg, seg_lo, valid, c0, x);
+            }
+        } else {
+            const int split = cid % sp.ksplit, tile = cid / sp.ksplit;
+            const int ldp = (sp.Np + 31) & ~31;          // partial row stride: whole 32-column groups
+            for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
+                uint32_t x[32];
+                tmem_ld32(lane_base + (uint32_t)(acc * sp.Np + c0), x);
+                tmem_wait_ld();
+                if (valid) {
+                    float4 *dst = reinterpret_cast<float4 *>(sp.ws_part + ((size_t)split * rows + row) * ldp + c0);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_float4(__uint_as_float(x[4 * c]), __uint_as_float(x[4 * c + 1]),
+                                             __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3]));
+                }
+            }
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            __shared__ int last_split;
+            if (threadIdx.x == 0) {
+                last_split = atomicAdd(sp.ws_count + tile, 1u) == (unsigned)(sp.ksplit - 1);
+                if (last_split) sp.ws_count[tile] = 0u;          // every split has arrived
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (last_split) {
+                __threadfence();
+                for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
+                    float sum[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) sum[c] = 0.f;
+                    if (valid)
+                        for (int s2 = 0; s2 < sp.ksplit; ++s2) {
+                            const float4 *src =
+                                reinterpret_cast<const float4 *>(sp.ws_part + ((size_t)s2 * rows + row) * ldp + c0);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const float4 v = __ldcg(src + c);
+                                sum[4 * c] += v.x;
+                                sum[4 * c + 1] += v.y;
+                                sum[4 * c + 2] += v.z;
+                                sum[4 * c + 3] += v.w;
+                            }
+                        }
+                    uint32_t x[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) x[c] = __float_as_uint(sum[c]);
+                    f(row, seg, seg_lo, valid, c0, x);
+                }
+            }
         }
         tc_fence_before();
         __syncwarp();

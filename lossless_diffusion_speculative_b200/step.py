@@ -104,6 +104,8 @@ class DecodeStep:
             self.w_qkv.append(tuple(
                 (torch.randn((n * D, Hd), generator=g, device=dev) * sc).to(dt)
                 for n in (Hq, Hkv, Hkv)))
+        self.qkv_ws = torch.zeros(ob.orthrus_qkv_workspace_size(B, K, Hd, Hq, Hkv, D), dtype=torch.uint8,
+                                  device=dev)
         self.project = True
 
     # -- the hot path, as launch sequences ---------------------------------
@@ -124,7 +126,7 @@ class DecodeStep:
     def _project(self, view, layer):
         wq, wk, wv = self.w_qkv[layer]
         ob.orthrus_qkv_project(self.x_all[view, layer], wq, wk, wv, self.ctx, self.q_all[view, layer],
-                               self.k_cache[layer], self.v_cache[layer], status=self.status)
+                               self.k_cache[layer], self.v_cache[layer], self.qkv_ws, status=self.status)
 
     def _fused_view(self, view):
         for layer in range(self.L):

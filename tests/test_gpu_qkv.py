@@ -43,8 +43,14 @@ def _gpu(x, wq, wk, wv, kc, vc, ctx, status=None):
     own = status is None
     if own:
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ob.orthrus_qkv_project(dev(x), dev(wq), dev(wk), dev(wv), torch.from_numpy(ctx).cuda(), q, tk, tv,
-                           status=status)
+    ws = torch.zeros(ob.orthrus_qkv_workspace_size(B, K, x.shape[2], Hq, kc.shape[1], kc.shape[3]),
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(2):                               # (the second call reuses the workspace)
+        ob.orthrus_qkv_project(dev(x), dev(wq), dev(wk), dev(wv), torch.from_numpy(ctx).cuda(), q, tk, tv,
+                               ws, status=status)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero().item()) == 0 or ob.orthrus_qkv_workspace_size(
+        B, K, x.shape[2], Hq, kc.shape[1], kc.shape[3]) > 4096   # (partials may stay)
     torch.cuda.synchronize()
     if own:
         assert int(status.item()) == 0

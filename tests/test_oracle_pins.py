@@ -576,3 +576,24 @@ def test_install_block_rows_places_the_tail_only():
             keep = np.r_[0:c, c + K:S]
             assert (k2[b, g, keep] == kc[b, g, keep]).all() and (v2[b, g, keep] == vc[b, g, keep]).all()
     assert (k2[2] == kc[2]).all() and (v2[2] == vc[2]).all()
+
+
+# --------------------------------------------------------------------------- prefill
+
+def test_ar_view_at_empty_context_is_causal_prefill_library():
+    """Causal prefill over S prompt tokens is the AR view with no committed
+    context and K = S: it matches the library's causal SDPA (torch, fp64)."""
+    rng = np.random.default_rng(60)
+    B, S, Hq, Hkv, D = 2, 11, 4, 2, 8
+    q = rng.standard_normal((B, S, Hq, D)).astype(np.float32)
+    kc = rng.standard_normal((B, Hkv, S + 3, D)).astype(np.float32)
+    vc = rng.standard_normal((B, Hkv, S + 3, D)).astype(np.float32)
+    out = oracle.attention(oracle.AR, q, kc, vc, np.zeros(B, np.int32))
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            qt = torch.from_numpy(q[b, :, h].astype(np.float64))[None]
+            kt = torch.from_numpy(kc[b, h // G, :S].astype(np.float64))[None]
+            vt = torch.from_numpy(vc[b, h // G, :S].astype(np.float64))[None]
+            ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)[0].numpy()
+            np.testing.assert_allclose(out[b, :, h], ref, rtol=1e-12, atol=1e-12)
