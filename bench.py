@@ -79,7 +79,29 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="time one entry of the configs block alone (a profiling aid) and print it")
     return ap.parse_args()
+
+
+def measure_one(label, dev, stream, hbm, iters):
+    """One entry of the configs block by its label."""
+    from lossless_diffusion_speculative_b200 import workloads as wl
+    for lab, name, order in CONFIG_SET:
+        if lab == label:
+            return measure_config(lab, wl.WORKLOADS[name], order, dev, stream, hbm, iters)
+    if label == "qwen3_8b_step_fused_qkv":
+        return measure_fused_step("qwen3_8b_step", dev, stream, hbm, iters)
+    for name in LM_HEAD_SET:
+        if label == "lm_head_consensus_" + name:
+            return measure_lm_head(name, dev, stream, hbm, iters)
+    for name, S in PREFILL_SET:
+        if label == f"prefill_{name}_S{S}":
+            return measure_prefill(name, S, dev, stream, tensor_peak()[0], iters)
+    for name in REJECT_SET:
+        if label == "rejection_verify_" + name:
+            return measure_rejection(name, dev, stream, hbm, iters)
+    raise SystemExit(f"--only: no configs entry named {label!r}")
 
 
 def peaks():
@@ -92,6 +114,16 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """Measured dense bf16 TFLOP/s (burst: a kernel timed on its own)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def kernel_hash():
     p = os.path.join(ROOT, "lossless_diffusion_speculative_b200", "csrc", "attn_tc.cu")
     with open(p, "rb") as f:
@@ -100,12 +132,13 @@ def kernel_hash():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (100 ms) of SM clock, power and throttle reasons,
-    from the first warm-up step to the end of the last GPU leg.  Samples whose
-    power draw shows the GPU busy count as "under load"."""
+    """nvidia-smi samples (100 ms) of SM clock, power, throttle reasons and GPU
+    utilisation, from the first warm-up step to the end of the last GPU leg.
+    Samples with the GPU at least half busy count as "under load"."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
@@ -140,18 +173,18 @@ class ClockSampler:
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
                 sm, smax, pw = float(parts[0]), float(parts[1]), float(parts[2])
+                util = float(parts[8])
             except ValueError:
                 continue
             active = {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}
-            rows.append((sm, smax, pw, active))
+            rows.append((sm, smax, pw, active, util))
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        idle = min(r[2] for r in rows)
-        load = [r for r in rows if r[2] >= idle + 100.0] or rows
+        load = [r for r in rows if r[4] >= 50.0] or rows
         reasons = sorted(set().union(*[r[3] for r in load]))
         return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": rows[-1][1],
                 "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
@@ -365,6 +398,54 @@ def measure_fused_step(name, dev, stream, hbm, iters, st=None):
     return out
 
 
+# ----------------------------------------------------------------------------- prefill
+PREFILL_SET = (("qwen3_8b_step", 4096), ("qwen3_8b_step", 16384))
+
+
+def measure_prefill(name, S, dev, stream, tf_peak, iters):
+    """orthrus_prefill_attn over one layer of an S-token prompt of the
+    workload's attention shape (batch 1): median µs, and the tensor throughput
+    on the causal attention's algorithmic flops, 4 * Hq * D * S (S + 1) / 2
+    (Q K^T and P V; the kernel's second P V term, which keeps the bf16
+    probabilities exact to 2^-14, is not counted)."""
+    import torch
+    from lossless_diffusion_speculative_b200 import binding as ob
+    from lossless_diffusion_speculative_b200 import workloads as wl
+
+    w = wl.WORKLOADS[name]
+    Hq, Hkv, D = w.Hq, w.Hkv, w.D
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 * w.cid + 94 + S)
+    sc = 1.0 / D ** 0.5
+    q = (torch.randn((1, S, Hq, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+    kc = (torch.randn((1, Hkv, S + 64, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+    vc = (torch.randn((1, Hkv, S + 64, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+    out = torch.empty((1, S, Hq, D), dtype=torch.float32, device=dev)
+    ws = torch.zeros(ob.orthrus_prefill_workspace_size(1, S, Hq, Hkv, D), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for it in range(3 + iters):
+            flush.zero_()
+            if it >= 3:
+                ev[it - 3][0].record()
+            ob.orthrus_prefill_attn(q, kc, vc, out, ws, status=status, stream=stream)
+            if it >= 3:
+                ev[it - 3][1].record()
+        torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"prefill: device status {int(status.item()):#x}")
+    us = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev])) * 1e3
+    flops = 4.0 * Hq * D * S * (S + 1) / 2
+    tf = flops / (us * 1e-6) / 1e12
+    return {"workload": name, "S": S, "Hq": Hq, "Hkv": Hkv, "D": D, "us_per_layer": us,
+            "tflops": tf, "frac_of_tensor_peak": tf / tf_peak, "iters": iters,
+            "kernel": "attn_tc_kernel (prompt chunks as AR-view blocks)",
+            "timing": "median of CUDA events per call; L2 flushed before each call"}
+
+
 # ----------------------------------------------------------------------------- fused LM head
 LM_HEAD_SET = ("qwen3_1p7b_layer", "qwen3_8b_step", "qwen3_4b_ragged", "qwen3_8b_long_k32")
 
@@ -455,7 +536,7 @@ def measure_rejection(name, dev, stream, hbm, iters):
     ur = torch.rand((B,), generator=g, device=dev)
     acc = torch.empty(B, dtype=torch.int32, device=dev)
     nxt = torch.empty(B, dtype=torch.int32, device=dev)
-    ws = torch.empty(ob.orthrus_rejection_workspace_size(B, K, V), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(ob.orthrus_rejection_workspace_size(B, K, V), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(iters)]
@@ -473,7 +554,7 @@ def measure_rejection(name, dev, stream, hbm, iters):
     gbs = nbytes / (us * 1e-6) / 1e9
     out = {"workload": name, "B": B, "K": K, "V": V, "us_per_call": us, "bytes": nbytes,
            "read_gbs": gbs, "frac_of_hbm": gbs / hbm, "mean_accepted": float(acc.float().mean()),
-           "iters": iters, "kernel": "rs_stats_kernel + rs_verify_kernel",
+           "iters": iters, "kernel": "rs_stats_kernel + rs_resid_kernel",
            "timing": "median of CUDA events per call; L2 flushed before each call"}
     del ar, dr, flush
     return out
@@ -500,6 +581,11 @@ def main():
     from lossless_diffusion_speculative_b200.step import DecodeStep
 
     torch.cuda.set_device(local)
+    if args.only:
+        dev = torch.device("cuda", local)
+        r = measure_one(args.only, dev, torch.cuda.Stream(device=dev), peaks()[0], args.steps)
+        print(json.dumps({"only": args.only, **r}), flush=True)
+        return
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -658,6 +744,10 @@ def main():
             for name in LM_HEAD_SET:
                 configs["lm_head_consensus_" + name] = measure_lm_head(name, dev, stream, hbm,
                                                                        CONFIG_ITERS)
+                torch.cuda.empty_cache()
+            tfp, _ = tensor_peak()
+            for name, S in PREFILL_SET:
+                configs[f"prefill_{name}_S{S}"] = measure_prefill(name, S, dev, stream, tfp, CONFIG_ITERS // 3)
                 torch.cuda.empty_cache()
             for name in REJECT_SET:
                 configs["rejection_verify_" + name] = measure_rejection(name, dev, stream, hbm,

@@ -89,9 +89,12 @@ typedef enum {
 
 /*
  * orthrus_attn_workspace_size — bytes of scratch orthrus_attn needs for these
- * sizes on the CURRENT device (a 1920-byte block of split-merge flags and counters, then
- * the split-KV partials: one fp32 [G*K, D] tile plus G*K log-sum-exp values
- * per (split unit, KV segment) boundary).  Independent of the context
+ * sizes on the CURRENT device: a 1920-byte block of split-merge flags and
+ * counters, then a 40960-byte cache of the per-CTA work split (each CTA's key
+ * range, stored with the shape and context lengths it was computed for, so a
+ * later call with the same lengths reads it back instead of recomputing it),
+ * then the split-KV partials: one fp32 [G*K, D] tile plus G*K log-sum-exp
+ * values per (split unit, KV segment) boundary.  Independent of the context
  * lengths.  Returns 0 for invalid sizes.
  */
 ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, int K,
@@ -124,10 +127,12 @@ ORTHRUS_API size_t orthrus_attn_workspace_size(int B, int Hq, int Hkv, int D, in
  *   workspace device scratch of at least orthrus_attn_workspace_size() bytes,
  *             16-byte aligned.  Zero-fill it once before its first use
  *             (cudaMemset): its leading counter block must be zero when a call
- *             starts, and every call that completes leaves it zero again (the
- *             rest is scratch, clobbered).  A call that ended with
- *             ORTHRUS_STATUS_TIMEOUT may leave counters set: zero it again.
- *             Calls that overlap on the device must not share it.
+ *             starts, and every call that completes leaves it zero again; the
+ *             work-split cache after it must hold zeros or what earlier calls
+ *             of this library wrote there (the rest is scratch, clobbered).  A
+ *             call that ended with ORTHRUS_STATUS_TIMEOUT may leave counters
+ *             set: zero it again.  Calls that overlap on the device must not
+ *             share it.
  *   status    optional device int32 (see ORTHRUS_STATUS_*).  A sequence whose
  *             ctx_lens[b] is negative or leaves no room for the block
  *             (ctx_lens[b] + K > S_max) sets ORTHRUS_STATUS_CAPACITY and its
@@ -217,7 +222,9 @@ ORTHRUS_API int orthrus_consensus(const float *logits, const int32_t *proposed, 
 
 /*
  * orthrus_rejection_workspace_size — scratch bytes for orthrus_rejection_verify
- * (one 16-byte (max, sum) pair of both views per vocabulary chunk per row).
+ * (one int32 counter per sequence, one 16-byte (max, sum) pair of both views per
+ * vocabulary chunk per row, and one float per 128-token tile of the vocabulary
+ * per sequence).
  */
 ORTHRUS_API size_t orthrus_rejection_workspace_size(int B, int K, int V);
 
@@ -246,7 +253,10 @@ ORTHRUS_API size_t orthrus_rejection_workspace_size(int B, int K, int V);
  *   u_resample   [B] fp32 uniform draws in [0, 1).
  *   temperature  > 0.
  *   workspace    >= orthrus_rejection_workspace_size(B, K, V) bytes, 16-byte
- *                aligned, clobbered.
+ *                aligned.  Zero-fill it once before its first use: its leading
+ *                per-sequence counters must be zero when a call starts, and
+ *                every call leaves them zero again (the rest is clobbered).
+ *                Calls that overlap on the device must not share it.
  * Supported: K <= ORTHRUS_MAX_BLOCK, V <= 262144, B * K <= 65535.
  * Numerics: fp32 with exp2 on the special-function unit; a decision whose
  * margin is within ~1e-6 relative of its threshold can differ from an exact

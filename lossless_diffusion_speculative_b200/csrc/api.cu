@@ -301,6 +301,23 @@ int orthrus_consensus(const float *logits, const int32_t *proposed, int B, int K
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 
+// Rejection workspace: [B] int32 counters (padded to 16 bytes), the chunk
+// statistics [B*K, splits] float4, then the residual tile sums [B, ntile].
+struct RejectLayout {
+    size_t count, stats, tiles, total;
+};
+
+static RejectLayout rejection_layout(int B, int K, int V, int splits)
+{
+    RejectLayout l;
+    const size_t ntile = ((size_t)V + 127) / 128;
+    l.count = 0;
+    l.stats = ((size_t)B * sizeof(int32_t) + 15) & ~(size_t)15;
+    l.tiles = l.stats + (size_t)B * K * splits * sizeof(float4);
+    l.total = l.tiles + (((size_t)B * ntile * sizeof(float) + 15) & ~(size_t)15);
+    return l;
+}
+
 size_t orthrus_rejection_workspace_size(int B, int K, int V)
 {
     if (B <= 0 || K <= 0 || V <= 0 || K > ORTHRUS_MAX_BLOCK) return 0;
@@ -308,7 +325,7 @@ size_t orthrus_rejection_workspace_size(int B, int K, int V)
     if (sms <= 0) return 0;
     int s, c;
     consensus_split(B, K, V, sms, &s, &c);
-    return (size_t)B * K * s * sizeof(float4);
+    return rejection_layout(B, K, V, s).total;
 }
 
 int orthrus_rejection_verify(const float *ar_logits, const float *draft_logits, const int32_t *proposed,
@@ -328,8 +345,16 @@ int orthrus_rejection_verify(const float *ar_logits, const float *draft_logits, 
     if (sms <= 0) return ORTHRUS_ERR_DEVICE;
     RejectArgs a;
     consensus_split(B, K, V, sms, &a.splits, &a.chunk);
-    const size_t need = (size_t)B * K * a.splits * sizeof(float4);
-    if (!workspace || workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+    const RejectLayout lay = rejection_layout(B, K, V, a.splits);
+    if (!workspace || workspace_bytes < lay.total) return ORTHRUS_ERR_WORKSPACE;
+    // residual pass: about one CTA per SM in total, at least one tile per warp
+    const int ntile = (V + 127) / 128;
+    int rs = (sms + B - 1) / B;
+    const int max_rs = (ntile + 7) / 8;
+    if (rs > max_rs) rs = max_rs;
+    if (rs < 1) rs = 1;
+    a.rtiles = (ntile + rs - 1) / rs;
+    a.rsplit = (ntile + a.rtiles - 1) / a.rtiles;
     a.ar = ar_logits;
     a.dr = draft_logits;
     a.proposed = proposed;
@@ -337,7 +362,10 @@ int orthrus_rejection_verify(const float *ar_logits, const float *draft_logits, 
     a.u_resample = u_resample;
     a.accepted = accepted_len;
     a.next_token = next_token;
-    a.ws = static_cast<float4 *>(workspace);
+    char *w = static_cast<char *>(workspace);
+    a.ws_count = reinterpret_cast<int32_t *>(w + lay.count);
+    a.ws = reinterpret_cast<float4 *>(w + lay.stats);
+    a.ws_tiles = reinterpret_cast<float *>(w + lay.tiles);
     a.status = status;
     a.B = B;
     a.K = K;

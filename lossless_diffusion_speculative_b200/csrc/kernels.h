@@ -151,8 +151,11 @@ struct RejectArgs {
     int32_t *accepted;
     int32_t *next_token;
     float4 *ws;                          // [B*K, splits] (max, sum) of both views, log2 units
+    float *ws_tiles;                     // [B, ceil(V / 128)] residual tile sums of the rejected row
+    int32_t *ws_count;                   // [B] CTAs done with the residual (zero between calls)
     int32_t *status;
     int B, K, V, splits, chunk;
+    int rsplit, rtiles;                  // residual pass: CTAs per sequence, tiles per CTA
     float c;                             // log2(e) / temperature
 };
 cudaError_t launch_rejection(const RejectArgs &p, cudaStream_t st);

@@ -15,12 +15,15 @@
 //   1. rs_stats: grid (splits, B*K).  Each CTA streams one vocabulary chunk of
 //      one row of both logit arrays (16-byte streaming loads) and reduces it to
 //      (max, sum of 2^(c x - max)) per array, c = log2(e) / T.
-//   2. rs_verify: one CTA per sequence merges the chunk statistics into each
-//      row's normalisers, takes the K accept decisions at once, keeps the first
-//      rejection a and, when a < K, streams row a of both arrays once more: each
-//      warp sums the residual over 128-element tiles, a block scan of the tile
-//      sums locates the tile holding u_resample * (total), and one warp scans
-//      that tile to the drawn token.
+//   2. rs_resid: grid (rsplit, B).  Every CTA of sequence b merges the chunk
+//      statistics into each row's normalisers and takes the K accept decisions
+//      (the same in every CTA), keeping the first rejection a.  When a < K,
+//      each CTA sums the residual of row a over its share of 128-element tiles
+//      (one warp per tile) into the workspace; the last CTA of the sequence to
+//      finish (a counter in the workspace) scans the tile sums to the tile
+//      holding u_resample * (total) and one warp scans that tile to the drawn
+//      token.  The tile sums and the scan are the same arithmetic in the same
+//      order whatever the number of CTAs, so the draw does not depend on it.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -140,16 +143,143 @@ __device__ __forceinline__ float block_excl_scan(float v, float *tmp, float *tot
     return tmp[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(kVerifyThreads) rs_verify_kernel(RejectArgs p)
+struct ResidShared {
+    Stat rp[ORTHRUS_MAX_BLOCK], rq[ORTHRUS_MAX_BLOCK];
+    float tile_sum[kMaxRejectTiles];
+    float scan_tmp[kVerifyThreads / 32];
+    float total;
+    int first_rej, tile_found, last;
+};
+
+// Residual mass of element v of one row (0 past the end).  The products are
+// explicitly rounded: the residual is the difference of two rounded
+// probabilities, exactly zero where the views agree, never an FMA-contracted
+// rounding error.
+struct RowMass {
+    const float *ar, *dr;
+    float c, mp, mq, ip, iq;
+    int V;
+    bool from_p;
+    __device__ __forceinline__ float operator()(int v) const
+    {
+        if (v >= V) return 0.f;
+        const float pv = __fmul_rn(fast_exp2(ar[v] * c - mp), ip);
+        if (from_p) return pv;
+        const float r = pv - __fmul_rn(fast_exp2(dr[v] * c - mq), iq);
+        return r > 0.f ? r : 0.f;
+    }
+};
+
+// Sum of tile k (128 elements: lane l holds elements 4l..4l+3, added in order,
+// then a butterfly over the lanes); every lane returns the sum.
+__device__ __forceinline__ float tile_mass(const RowMass &mass, int k, int lane)
 {
-    const int b = blockIdx.x;
+    const int v0 = k * kTileElems + lane * 4;
+    float s = mass(v0) + mass(v0 + 1) + mass(v0 + 2) + mass(v0 + 3);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// Inverse-CDF search over the row's tile sums (in shared memory): the token
+// whose cumulative mass first exceeds u * total.  Returns false (nothing
+// written) when the total is not positive.  Called by the whole block.
+__device__ bool draw_from_tiles(const RejectArgs &p, const RowMass &mass, ResidShared &sh, int ntile, int b,
+                                int a)
+{
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __shared__ Stat rp[ORTHRUS_MAX_BLOCK], rq[ORTHRUS_MAX_BLOCK];
-    __shared__ int first_rej;
-    __shared__ float tile_sum[kMaxRejectTiles];
-    __shared__ float scan_tmp[kVerifyThreads / 32];
-    __shared__ float total;
-    __shared__ int tile_found;
+    // tiles in contiguous runs per thread, then a block scan of the runs
+    const int per = (ntile + kVerifyThreads - 1) / kVerifyThreads;
+    const int t0 = threadIdx.x * per, t1 = t0 + per < ntile ? t0 + per : ntile;
+    float run = 0.f;
+    for (int k = t0; k < t1; ++k) run += sh.tile_sum[k];
+    const float pre = block_excl_scan(run, sh.scan_tmp, &sh.total);
+    const float R = sh.total;
+    if (!(R > 0.f)) return false;
+    const float target = p.u_resample[b] * R;
+    if (threadIdx.x == 0) sh.tile_found = -1;
+    __syncthreads();
+    // the run holding the target (the last nonempty one if rounding put it past the end)
+    float acc = pre;
+    int kt = -1;
+    for (int k = t0; k < t1; ++k) {
+        if (sh.tile_sum[k] > 0.f) kt = k;
+        if (sh.tile_sum[k] > 0.f && target < acc + sh.tile_sum[k]) break;
+        acc += sh.tile_sum[k];
+    }
+    const bool holds = t0 < t1 && pre <= target && (target < pre + run || threadIdx.x == kVerifyThreads - 1 ||
+                                                    t1 == ntile);
+    if (holds && kt >= 0) atomicMax(&sh.tile_found, kt);
+    __syncthreads();
+    int k = sh.tile_found;
+    if (k < 0) {                                      // (rounding: fall back to the last nonempty tile)
+        if (threadIdx.x == 0)
+            for (int j = ntile - 1; j >= 0; --j)
+                if (sh.tile_sum[j] > 0.f) {
+                    sh.tile_found = j;
+                    break;
+                }
+        __syncthreads();
+        k = sh.tile_found;
+    }
+    // prefix of the tiles before k (same order as the runs), then one warp scans tile k
+    if (warp == 0 && k >= 0) {
+        float before = 0.f;
+        for (int j = lane; j < k; j += 32) before += sh.tile_sum[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+        const int v0 = k * kTileElems + lane * 4;
+        const float m0 = mass(v0), m1 = mass(v0 + 1), m2 = mass(v0 + 2), m3 = mass(v0 + 3);
+        const float own = m0 + m1 + m2 + m3;
+        float incl = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const float t = target - before;              // position inside tile k
+        const float ex = incl - own;
+        const unsigned in = __ballot_sync(0xffffffffu, own > 0.f && t < incl);
+        int pick = -1;
+        if (in) {
+            const int l = __ffs(in) - 1;
+            if (lane == l) {
+                float c = ex;
+                pick = v0 + 3;
+                const float ms[4] = {m0, m1, m2, m3};
+                int last_nz = -1;
+                for (int e = 0; e < 4; ++e) {
+                    if (ms[e] > 0.f) last_nz = v0 + e;
+                    if (ms[e] > 0.f && t < c + ms[e]) {
+                        pick = v0 + e;
+                        last_nz = -2;
+                        break;
+                    }
+                    c += ms[e];
+                }
+                if (last_nz >= 0) pick = last_nz;
+            }
+            pick = __shfl_sync(0xffffffffu, pick, l);
+        } else {
+            // the target lies at or past the tile's end: the tile's last nonzero element
+            const unsigned nz = __ballot_sync(0xffffffffu, own > 0.f);
+            const int l = 31 - __clz(nz);
+            if (lane == l) pick = m3 > 0.f ? v0 + 3 : m2 > 0.f ? v0 + 2 : m1 > 0.f ? v0 + 1 : v0;
+            pick = __shfl_sync(0xffffffffu, pick, l);
+        }
+        if (lane == 0) {
+            p.accepted[b] = a;
+            p.next_token[b] = pick;
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kVerifyThreads) rs_resid_kernel(RejectArgs p)
+{
+    const int b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __shared__ ResidShared sh;
     // ---- each row's normalisers from its chunk statistics
     for (int i = warp; i < p.K; i += kVerifyThreads / 32) {
         const float4 *w = p.ws + ((size_t)b * p.K + i) * p.splits;
@@ -162,11 +292,11 @@ __global__ void __launch_bounds__(kVerifyThreads) rs_verify_kernel(RejectArgs p)
         u = warp_stat(u);
         v = warp_stat(v);
         if (lane == 0) {
-            rp[i] = u;
-            rq[i] = v;
+            sh.rp[i] = u;
+            sh.rq[i] = v;
         }
     }
-    if (threadIdx.x == 0) first_rej = p.K;
+    if (threadIdx.x == 0) sh.first_rej = p.K;
     __syncthreads();
     // ---- every slot's accept decision; the first rejection wins
     for (int i = threadIdx.x; i < p.K; i += kVerifyThreads) {
@@ -174,137 +304,65 @@ __global__ void __launch_bounds__(kVerifyThreads) rs_verify_kernel(RejectArgs p)
         const int x = p.proposed[row];
         bool keep = false;
         if (x >= 0 && x < p.V) {
-            const float px = fast_exp2(p.ar[row * p.V + x] * p.c - rp[i].m) / rp[i].l;
-            const float qx = fast_exp2(p.dr[row * p.V + x] * p.c - rq[i].m) / rq[i].l;
+            const float px = fast_exp2(p.ar[row * p.V + x] * p.c - sh.rp[i].m) / sh.rp[i].l;
+            const float qx = fast_exp2(p.dr[row * p.V + x] * p.c - sh.rq[i].m) / sh.rq[i].l;
             keep = p.u_accept[row] * qx < px;
         }
-        if (!keep) atomicMin(&first_rej, i);
+        if (!keep) atomicMin(&sh.first_rej, i);
     }
     __syncthreads();
-    const int a = first_rej;
+    const int a = sh.first_rej;
     if (a == p.K) {
-        if (threadIdx.x == 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
             p.accepted[b] = p.K;
             p.next_token[b] = p.proposed[(size_t)b * p.K + p.K - 1];
         }
         return;
     }
-    // ---- draw from the residual of row a
+    // ---- this CTA's share of the residual tile sums of row a
     const size_t row = (size_t)b * p.K + a;
-    const float *ar = p.ar + row * p.V, *dr = p.dr + row * p.V;
-    const Stat sp = rp[a], sq = rq[a];
-    const float ip = 1.f / sp.l, iq = 1.f / sq.l;
+    RowMass mass;
+    mass.ar = p.ar + row * p.V;
+    mass.dr = p.dr + row * p.V;
+    mass.c = p.c;
+    mass.mp = sh.rp[a].m;
+    mass.mq = sh.rq[a].m;
+    mass.ip = 1.f / sh.rp[a].l;
+    mass.iq = 1.f / sh.rq[a].l;
+    mass.V = p.V;
+    mass.from_p = false;
     const int ntile = (p.V + kTileElems - 1) / kTileElems;
-    for (int pass = 0; pass < 2; ++pass) {
-        const bool from_p = pass == 1;                // the residual was empty: draw from p
-        // (explicitly rounded products: the residual is the difference of two
-        // rounded probabilities, exactly zero where the views agree, never an
-        // FMA-contracted rounding error)
-        auto mass = [&](int v) -> float {
-            if (v >= p.V) return 0.f;
-            const float pv = __fmul_rn(fast_exp2(ar[v] * p.c - sp.m), ip);
-            if (from_p) return pv;
-            const float r = pv - __fmul_rn(fast_exp2(dr[v] * p.c - sq.m), iq);
-            return r > 0.f ? r : 0.f;
-        };
-        for (int k = warp; k < ntile; k += kVerifyThreads / 32) {
-            const int v0 = k * kTileElems + lane * 4;
-            float s = mass(v0) + mass(v0 + 1) + mass(v0 + 2) + mass(v0 + 3);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) tile_sum[k] = s;
-        }
-        __syncthreads();
-        // tiles in contiguous runs per thread, then a block scan of the runs
-        const int per = (ntile + kVerifyThreads - 1) / kVerifyThreads;
-        const int t0 = threadIdx.x * per, t1 = t0 + per < ntile ? t0 + per : ntile;
-        float run = 0.f;
-        for (int k = t0; k < t1; ++k) run += tile_sum[k];
-        const float pre = block_excl_scan(run, scan_tmp, &total);
-        const float R = total;
-        if (R <= 0.f) {
-            if (pass == 0) continue;                  // empty residual: draw from p
-        }
-        const float target = p.u_resample[b] * R;
-        if (threadIdx.x == 0) tile_found = -1;
-        __syncthreads();
-        // the run holding the target (the last nonempty one if rounding put it past the end)
-        float acc = pre;
-        int kt = -1;
-        for (int k = t0; k < t1; ++k) {
-            if (tile_sum[k] > 0.f) kt = k;
-            if (tile_sum[k] > 0.f && target < acc + tile_sum[k]) break;
-            acc += tile_sum[k];
-        }
-        const bool holds = t0 < t1 && pre <= target && (target < pre + run || threadIdx.x == kVerifyThreads - 1 ||
-                                                        t1 == ntile);
-        if (holds && kt >= 0) atomicMax(&tile_found, kt);
-        __syncthreads();
-        int k = tile_found;
-        if (k < 0) {                                  // (rounding: fall back to the last nonempty tile)
-            if (threadIdx.x == 0)
-                for (int j = ntile - 1; j >= 0; --j)
-                    if (tile_sum[j] > 0.f) {
-                        tile_found = j;
-                        break;
-                    }
-            __syncthreads();
-            k = tile_found;
-        }
-        // prefix of the tiles before k (same order as the runs), then one warp scans tile k
-        if (warp == 0 && k >= 0) {
-            float before = 0.f;
-            for (int j = lane; j < k; j += 32) before += tile_sum[j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
-            const int v0 = k * kTileElems + lane * 4;
-            const float m0 = mass(v0), m1 = mass(v0 + 1), m2 = mass(v0 + 2), m3 = mass(v0 + 3);
-            const float own = m0 + m1 + m2 + m3;
-            float incl = own;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += u;
-            }
-            const float t = target - before;          // position inside tile k
-            const float ex = incl - own;
-            const unsigned in = __ballot_sync(0xffffffffu, own > 0.f && t < incl);
-            int pick = -1;
-            if (in) {
-                const int l = __ffs(in) - 1;
-                if (lane == l) {
-                    float c = ex;
-                    pick = v0 + 3;
-                    const float ms[4] = {m0, m1, m2, m3};
-                    int last_nz = -1;
-                    for (int e = 0; e < 4; ++e) {
-                        if (ms[e] > 0.f) last_nz = v0 + e;
-                        if (ms[e] > 0.f && t < c + ms[e]) {
-                            pick = v0 + e;
-                            last_nz = -2;
-                            break;
-                        }
-                        c += ms[e];
-                    }
-                    if (last_nz >= 0) pick = last_nz;
-                }
-                pick = __shfl_sync(0xffffffffu, pick, l);
-            } else {
-                // the target lies at or past the tile's end: the tile's last nonzero element
-                const unsigned nz = __ballot_sync(0xffffffffu, own > 0.f);
-                const int l = 31 - __clz(nz);
-                if (lane == l) {
-                    pick = m3 > 0.f ? v0 + 3 : m2 > 0.f ? v0 + 2 : m1 > 0.f ? v0 + 1 : v0;
-                }
-                pick = __shfl_sync(0xffffffffu, pick, l);
-            }
-            if (lane == 0) {
-                p.accepted[b] = a;
-                p.next_token[b] = pick;
-            }
-        }
-        break;
+    float *tiles = p.ws_tiles + (size_t)b * ntile;
+    const int k0 = blockIdx.x * p.rtiles;
+    const int k1 = k0 + p.rtiles < ntile ? k0 + p.rtiles : ntile;
+    for (int k = k0 + warp; k < k1; k += kVerifyThreads / 32) {
+        const float s = tile_mass(mass, k, lane);
+        if (lane == 0) tiles[k] = s;
     }
+    // ---- the last CTA of the sequence draws
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int done = atomicAdd(p.ws_count + b, 1);
+        sh.last = done == (int)gridDim.x - 1;
+        if (sh.last) {
+            __threadfence();
+            p.ws_count[b] = 0;                        // left zero for the next call
+        }
+    }
+    __syncthreads();
+    if (!sh.last) return;
+    for (int k = threadIdx.x; k < ntile; k += kVerifyThreads) sh.tile_sum[k] = __ldcg(tiles + k);
+    __syncthreads();
+    if (draw_from_tiles(p, mass, sh, ntile, b, a)) return;
+    // the residual is empty (p and q agree on row a): draw from p, in this CTA alone
+    mass.from_p = true;
+    for (int k = warp; k < ntile; k += kVerifyThreads / 32) {
+        const float s = tile_mass(mass, k, lane);
+        if (lane == 0) sh.tile_sum[k] = s;
+    }
+    __syncthreads();
+    draw_from_tiles(p, mass, sh, ntile, b, a);
 }
 
 }  // namespace
@@ -315,7 +373,7 @@ cudaError_t launch_rejection(const RejectArgs &p, cudaStream_t st)
     rs_stats_kernel<<<g1, kStatsThreads, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    rs_verify_kernel<<<p.B, kVerifyThreads, 0, st>>>(p);
+    rs_resid_kernel<<<dim3(p.rsplit, p.B), kVerifyThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

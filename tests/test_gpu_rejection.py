@@ -31,11 +31,12 @@ def _gpu(ar, dr, prop, ua, ur, T):
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     acc = torch.full((B,), -7, dtype=torch.int32, device="cuda")
     nxt = torch.full((B,), -7, dtype=torch.int32, device="cuda")
-    ws = torch.empty(ob.orthrus_rejection_workspace_size(B, K, V), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(ob.orthrus_rejection_workspace_size(B, K, V), dtype=torch.uint8, device="cuda")
     ob.orthrus_rejection_verify(dev(ar.astype(np.float32)), dev(dr.astype(np.float32)),
                                 dev(prop.astype(np.int32)), dev(ua.astype(np.float32)),
                                 dev(ur.astype(np.float32)), T, acc, nxt, ws)
     torch.cuda.synchronize()
+    assert int(ws[:4 * B].count_nonzero().item()) == 0, "per-sequence counters not left zero"
     return acc.cpu().numpy(), nxt.cpu().numpy()
 
 
