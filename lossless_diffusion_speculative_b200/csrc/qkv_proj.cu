@@ -35,6 +35,42 @@ namespace qkv {
 
 using namespace sm100;
 
+// Shared-memory table of the epilogue: per token row t = b * K + i, the cache
+// row of its key and value in KV head 0, (b * Hkv) * S_max + ctx_b + i, or -1
+// when sequence b has no room for its block.
+constexpr uint32_t kTokBytes = kMaxLmRows * sizeof(long long);
+
+// The epilogue's store of one 32-token group of one output feature (a warp's
+// 32 lanes hold 32 consecutive features: every store of the warp is 64
+// contiguous bytes).
+struct QkvStore {
+    __nv_bfloat16 *q, *kc, *vc;
+    const long long *tokrow;
+    int qrow, D, S_max, BK;
+    __device__ __forceinline__ void operator()(int row, int seg, int seg_lo, bool valid, int c0,
+                                               const uint32_t (&x)[32]) const
+    {
+        if (!valid) return;
+        const int f = row - seg_lo;                                   // feature in its segment
+        if (seg == 0) {
+            __nv_bfloat16 *dst = q + f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+                if (c0 + c < BK) dst[(size_t)(c0 + c) * qrow] = __float2bfloat16_rn(__uint_as_float(x[c]));
+        } else {
+            const int g = f / D, d = f - g * D;                       // KV head, dim
+            __nv_bfloat16 *dst = (seg == 1 ? kc : vc) + (size_t)g * S_max * D + d;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                if (c0 + c < BK) {
+                    const long long r = tokrow[c0 + c];
+                    if (r >= 0) dst[r * D] = __float2bfloat16_rn(__uint_as_float(x[c]));
+                }
+            }
+        }
+    }
+};
+
 template <int CPS, bool SPLITK>
 __global__ void __launch_bounds__(sg::kThreads, 1)
     qkv_proj_kernel(const __grid_constant__ sg::Maps mp, const QkvArgs p)
@@ -43,7 +79,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     const sg::Shape &sp = p.shape;
     sg::Smem sm;
     pdl_trigger();
-    sg::prologue(sm, smem_raw, sp, CPS, 0, mp);
+    sg::prologue(sm, smem_raw, sp, CPS, kTokBytes, mp);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     tc_fence_before();
     __syncthreads();
@@ -53,39 +89,26 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     // ---- everything below may read what earlier kernels wrote
     pdl_wait();
     const int cid = blockIdx.x, grid = gridDim.x;
-    if (cid == 0)
-        for (int b = threadIdx.x; b < p.B; b += sg::kThreads) {
-            const int c = p.ctx_lens[b];
-            if (c < 0 || (int64_t)c + p.K > p.S_max) raise_status(sp.status, ORTHRUS_STATUS_CAPACITY);
-        }
     if (warp < 4) {
-        __nv_bfloat16 *q = static_cast<__nv_bfloat16 *>(p.q_out);
-        __nv_bfloat16 *kc = static_cast<__nv_bfloat16 *>(p.k_cache);
-        __nv_bfloat16 *vc = static_cast<__nv_bfloat16 *>(p.v_cache);
-        const int qrow = p.Hq * p.D, D = p.D, K = p.K, Hkv = p.Hkv, S_max = p.S_max, BK = sp.BK;
-        const int32_t *ctx_lens = p.ctx_lens;
-        sg::epilogue_tiles<SPLITK>(sm, sp, cid, grid, tmem, CPS,
-                           [=](int row, int seg, int seg_lo, bool valid, int c0, const uint32_t (&x)[32]) {
-                               if (!valid) return;
-                               const int f = row - seg_lo;                   // feature in its segment
-                               const int g = f / D, d = f - g * D;           // (k, v: KV head, dim)
-                               __nv_bfloat16 *cache = seg == 1 ? kc : vc;
-#pragma unroll
-                               for (int c = 0; c < 32; ++c) {
-                                   const int t = c0 + c;
-                                   if (t < BK) {
-                                       const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(x[c]));
-                                       if (seg == 0) {
-                                           q[(size_t)t * qrow + f] = v;
-                                       } else {
-                                           const int b = t / K, i = t - b * K;
-                                           const int ctx = __ldg(ctx_lens + b);
-                                           if (ctx >= 0 && (int64_t)ctx + K <= S_max)
-                                               cache[(((size_t)b * Hkv + g) * S_max + ctx + i) * D + d] = v;
-                                       }
-                                   }
-                               }
-                           });
+        long long *tokrow = reinterpret_cast<long long *>(sm.extra());
+        for (int t = threadIdx.x; t < sp.BK; t += 128) {
+            const int b = t / p.K, i = t - b * p.K;
+            const int c = p.ctx_lens[b];
+            const bool room = c >= 0 && (int64_t)c + p.K <= p.S_max;
+            if (!room && i == 0 && cid == 0) raise_status(sp.status, ORTHRUS_STATUS_CAPACITY);
+            tokrow[t] = room ? (long long)b * p.Hkv * p.S_max + c + i : -1ll;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        QkvStore st;
+        st.q = static_cast<__nv_bfloat16 *>(p.q_out);
+        st.kc = static_cast<__nv_bfloat16 *>(p.k_cache);
+        st.vc = static_cast<__nv_bfloat16 *>(p.v_cache);
+        st.tokrow = tokrow;
+        st.qrow = p.Hq * p.D;
+        st.D = p.D;
+        st.S_max = p.S_max;
+        st.BK = sp.BK;
+        sg::epilogue_tiles<SPLITK>(sm, sp, cid, grid, tmem, CPS, st);
     } else if (warp == 4) {
         if (lane == 0) sg::producer<CPS>(sm, sp, mp, cid, grid);
         __syncwarp();
@@ -226,7 +249,7 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
     sp.ws_part = static_cast<float *>(workspace);
     sp.ws_count = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + qp.part_bytes);
     const int cps = qp.cps;
-    const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, 0);
+    const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, qkv::kTokBytes);
 
     sg::Maps mp;
     if (!sg::encode_w(mp, 0, w_q, Hq * D, hidden) || !sg::encode_w(mp, 1, w_k, Hkv * D, hidden) ||

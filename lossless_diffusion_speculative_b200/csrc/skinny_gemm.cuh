@@ -43,6 +43,7 @@ constexpr int kMaxStages = 12;
 constexpr uint32_t kRingBudget = 200 * 1024;
 constexpr int kTmemCols = 512;
 constexpr int kMaxSegs = 3;
+constexpr int kSumBatch = 4;                        // split-K partials loaded at once by the last split
 
 enum : int {
     B_FULL = 0,
@@ -297,33 +298,61 @@ __device__ __forceinline__ bool epilogue_tiles(const Smem &sm, const Shape &sp, 
                                              __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3]));
                 }
             }
-            __threadfence();
+            // The barrier orders the four warps' partial stores before thread
+            // 0's release; its acquire, then the barrier, orders every other
+            // split's partial before this CTA's loads when it is the last.
             asm volatile("bar.sync 1, 128;" ::: "memory");
             __shared__ int last_split;
             if (threadIdx.x == 0) {
-                last_split = atomicAdd(sp.ws_count + tile, 1u) == (unsigned)(sp.ksplit - 1);
+                unsigned int old;
+                asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+                             : "=r"(old)
+                             : "l"(sp.ws_count + tile)
+                             : "memory");
+                last_split = old == (unsigned)(sp.ksplit - 1);
                 if (last_split) sp.ws_count[tile] = 0u;          // every split has arrived
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (last_split) {
-                __threadfence();
                 for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
+                    // this split's own partial again from TMEM; the others' from
+                    // L2, kSumBatch at a time; summed in split order from zero, so the
+                    // result does not depend on which split finished last
+                    uint32_t own[32];
+                    tmem_ld32(lane_base + (uint32_t)(acc * sp.Np + c0), own);
+                    tmem_wait_ld();
                     float sum[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) sum[c] = 0.f;
-                    if (valid)
-                        for (int s2 = 0; s2 < sp.ksplit; ++s2) {
-                            const float4 *src =
-                                reinterpret_cast<const float4 *>(sp.ws_part + ((size_t)s2 * rows + row) * ldp + c0);
+                    for (int s2 = 0; s2 < sp.ksplit; s2 += kSumBatch) {
+                        // up to kSumBatch partials' loads in flight at once
+                        float4 v[kSumBatch][8];
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const float4 v = __ldcg(src + c);
-                                sum[4 * c] += v.x;
-                                sum[4 * c + 1] += v.y;
-                                sum[4 * c + 2] += v.z;
-                                sum[4 * c + 3] += v.w;
+                        for (int u = 0; u < kSumBatch; ++u) {
+                            const int su = s2 + u;
+                            const float4 *src =
+                                reinterpret_cast<const float4 *>(sp.ws_part + ((size_t)su * rows + row) * ldp + c0);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                v[u][c] = !valid || su >= sp.ksplit ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                          : su != split
+                                              ? __ldcg(src + c)
+                                              : make_float4(__uint_as_float(own[4 * c]), __uint_as_float(own[4 * c + 1]),
+                                                            __uint_as_float(own[4 * c + 2]), __uint_as_float(own[4 * c + 3]));
+                        }
+#pragma unroll
+                        for (int u = 0; u < kSumBatch; ++u) {
+                            if (s2 + u < sp.ksplit) {
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) {
+                                    sum[4 * c] += v[u][c].x;
+                                    sum[4 * c + 1] += v[u][c].y;
+                                    sum[4 * c + 2] += v[u][c].z;
+                                    sum[4 * c + 3] += v[u][c].w;
+                                }
                             }
                         }
+                    }
                     uint32_t x[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) x[c] = __float_as_uint(sum[c]);
