@@ -54,7 +54,7 @@ REF_BUDGET_S = 150.0                # reference arm: timed CPU seconds per run
 # DRAM traffic of one attn_tc_kernel launch on the headline workload, from the
 # ncu capture summarised in profiles/ (bytes read + written), keyed by the hash
 # of the kernel source it was taken on; reported as null once the source changes.
-NCU_TRAFFIC = {("qwen3_8b_step", "3a5dfd49b7df8d12"): 34.05e6}
+NCU_TRAFFIC = {("qwen3_8b_step", "5fa3835a6b71460c"): 34.09e6}
 
 # The workloads of the configs block: (label, workload, order).  The 36-layer
 # step in its specified per-layer order (DIFF then AR per layer) is timed in
@@ -95,6 +95,9 @@ def measure_one(label, dev, stream, hbm, iters):
     for name in LM_HEAD_SET:
         if label == "lm_head_consensus_" + name:
             return measure_lm_head(name, dev, stream, hbm, iters)
+    for name in QKV_SET:
+        if label == "qkv_projection_" + name:
+            return measure_qkv(name, dev, stream, hbm, iters)
     for name, S in PREFILL_SET:
         if label == f"prefill_{name}_S{S}":
             return measure_prefill(name, S, dev, stream, tensor_peak()[0], iters)
@@ -396,6 +399,58 @@ def measure_fused_step(name, dev, stream, hbm, iters, st=None):
                 "verified_tokens_per_s_at_expected": st.tokens_per_step_expected() / (step_us * 1e-6),
                 "timing": "median of per-segment CUDA events over graph replays (inputs larger than L2)"})
     return out
+
+
+# ----------------------------------------------------------------------------- QKV projection
+QKV_SET = ("qwen3_1p7b_layer", "qwen3_8b_step", "qwen3_4b_ragged")
+
+
+def measure_qkv(name, dev, stream, hbm, iters):
+    """orthrus_qkv_project for one layer and one view of the workload (its
+    width, heads and batch; the block's key and value rows written into a
+    cache of context 8192): median µs per call with L2 flushed before each,
+    and the weight-read bandwidth (the stacked [Hq + 2 Hkv] * D x hidden bf16
+    weights are the algorithmic traffic; the block's hidden states and outputs
+    are < 2 % of it at B * K = 32)."""
+    import torch
+    from lossless_diffusion_speculative_b200 import binding as ob
+    from lossless_diffusion_speculative_b200 import workloads as wl
+
+    w = wl.WORKLOADS[name]
+    B, K, hidden, Hq, Hkv, D = w.B, w.K, w.hidden, w.Hq, w.Hkv, w.D
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 * w.cid + 93)
+    x = torch.randn((B, K, hidden), generator=g, device=dev).to(torch.bfloat16)
+    wts = [(torch.randn((n * D, hidden), generator=g, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+           for n in (Hq, Hkv, Hkv)]
+    ctx = 8192
+    kc = torch.zeros((B, Hkv, ctx + 2 * K, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    ctx_lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    q = torch.empty((B, K, Hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(ob.orthrus_qkv_workspace_size(B, K, hidden, Hq, Hkv, D), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for it in range(3 + iters):
+            flush.zero_()
+            if it >= 3:
+                ev[it - 3][0].record()
+            ob.orthrus_qkv_project(x, *wts, ctx_lens, q, kc, vc, ws, status=status, stream=stream)
+            if it >= 3:
+                ev[it - 3][1].record()
+        torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"qkv projection: device status {int(status.item()):#x}")
+    us = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev])) * 1e3
+    wb = sum(t.numel() * 2 for t in wts)
+    gbs = wb / (us * 1e-6) / 1e9
+    return {"workload": name, "B": B, "K": K, "hidden": hidden, "Hq": Hq, "Hkv": Hkv, "D": D,
+            "us_per_call": us, "weight_bytes": wb, "weight_read_gbs": gbs, "frac_of_hbm": gbs / hbm,
+            "iters": iters, "kernel": "qkv_proj_kernel (tcgen05 skinny GEMM, split-K, cache-row store)",
+            "timing": "median of CUDA events per call; L2 flushed before each call"}
 
 
 # ----------------------------------------------------------------------------- prefill
@@ -744,6 +799,9 @@ def main():
             for name in LM_HEAD_SET:
                 configs["lm_head_consensus_" + name] = measure_lm_head(name, dev, stream, hbm,
                                                                        CONFIG_ITERS)
+                torch.cuda.empty_cache()
+            for name in QKV_SET:
+                configs["qkv_projection_" + name] = measure_qkv(name, dev, stream, hbm, CONFIG_ITERS)
                 torch.cuda.empty_cache()
             tfp, _ = tensor_peak()
             for name, S in PREFILL_SET:

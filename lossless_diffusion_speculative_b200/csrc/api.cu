@@ -157,12 +157,13 @@ int attn_call(orthrus_view view, orthrus_dtype dtype, const void *q, const void 
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 
-// Chunked prefill: prompt chunk c of sequence s runs as call sequence
-// s * nch + c, an AR-view block of kc tokens after c * kc context tokens.
+// Chunked prefill: call sequence s * nch + j is prompt chunk
+// c = prefill_chunk_of(j, nch) of sequence s, an AR-view block of kc tokens
+// after c * kc context tokens.
 __global__ void prefill_ctx_kernel(int32_t *ctx, int n, int nch, int kc, int offset)
 {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b < n) ctx[b] = (b % nch) * kc + offset;
+    if (b < n) ctx[b] = prefill_chunk_of(b % nch, nch) * kc + offset;
 }
 
 int prefill_chunk(int G)

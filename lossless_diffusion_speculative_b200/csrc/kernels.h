@@ -28,17 +28,31 @@ struct AttnArgs {
     int min_keys;        // smallest key range worth a CTA
     // Sequence b of the call reads the cache of sequence b / cache_div and the
     // query / output rows from q_row0(b); a decode call has cache_div = 1 and
-    // q_seq_rows = K (rows b * K).  Chunked prefill runs prompt chunk c of
-    // sequence s as call sequence s * cache_div + c.
+    // q_seq_rows = K (rows b * K).  Chunked prefill runs prompt chunk
+    // prefill_chunk_of(j, cache_div) of sequence s as call sequence
+    // s * cache_div + j.
     int cache_div;
     int q_seq_rows;
     __host__ __device__ __forceinline__ int cache_seq(int b) const { return cache_div == 1 ? b : b / cache_div; }
-    __host__ __device__ __forceinline__ size_t q_row0(int b) const
-    {
-        return cache_div == 1 ? (size_t)b * q_seq_rows
-                              : (size_t)(b / cache_div) * q_seq_rows + (size_t)(b % cache_div) * K;
-    }
+    __host__ __device__ __forceinline__ size_t q_row0(int b) const;
 };
+
+// Order of a prompt's chunks in a chunked-prefill call: shortest and longest
+// alternate (0, n-1, 1, n-2, ...), so that the equal key ranges of the work
+// split each hold a few short segments instead of one range holding all of
+// them (every segment costs a fixed query load and epilogue on top of its
+// keys).
+__host__ __device__ __forceinline__ int prefill_chunk_of(int j, int n)
+{
+    return (j & 1) ? n - 1 - (j >> 1) : (j >> 1);
+}
+
+__host__ __device__ __forceinline__ size_t AttnArgs::q_row0(int b) const
+{
+    return cache_div == 1 ? (size_t)b * q_seq_rows
+                          : (size_t)(b / cache_div) * q_seq_rows +
+                                (size_t)prefill_chunk_of(b % cache_div, cache_div) * K;
+}
 
 // Workspace layout shared by the attention paths: a fixed block of flags and
 // counters used by the tensor-core path's in-kernel split merge (zero before
