@@ -32,9 +32,10 @@
 // (+ TMEM allocation), warp 6 PV MMAs (an MMA issue blocks its thread while
 // the tensor pipe is busy, so S and PV each get a thread of their own).
 // S is triple-buffered in TMEM (3 x 128 columns) next to the O accumulator
-// (128 columns); the query tile, two K stages and four V stages sit in shared
-// memory; after a piece the rings stage the output rows for their bulk
-// copies.
+// (128 columns); the query tile, three K stages and three V stages sit in
+// shared memory (under a full HBM stream a K tile lands ~2 us after its
+// request, longer than two tile periods); after a piece the rings stage the
+// output rows for their bulk copies.
 // Launched with programmatic dependent launch: barrier setup, TMEM allocation
 // and descriptor prefetch overlap the previous kernel; nothing an earlier
 // kernel may write (ctx_lens, queries, cache, workspace) is read before
@@ -57,8 +58,8 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                  // M of every MMA (G*K <= 128 used)
-constexpr int kKStages = 2;
-constexpr int kVStages = 4;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
 constexpr int kSBuf = 3;                    // S can run two tiles ahead of PV
 constexpr int kThreads = 224;
 constexpr int kBoxKeys = 64;
