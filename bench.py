@@ -302,7 +302,7 @@ def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
     replays, L2 flushed before every attention segment (outside the events).
     `st` reuses an existing DecodeStep of the same workload."""
     import torch
-    from lossless_diffusion_speculative_b200.step import DecodeStep
+    from lossless_diffusion_speculative_b200.step import DecodeStep, layer_groups
 
     if st is None:
         st = DecodeStep(w, order=order, device=dev)
@@ -355,7 +355,7 @@ def measure_fused_step(name, dev, stream, hbm, iters, st=None):
     alone (same launches, no attention) for their weight-read bandwidth."""
     import torch
     from lossless_diffusion_speculative_b200 import workloads as wl
-    from lossless_diffusion_speculative_b200.step import DecodeStep
+    from lossless_diffusion_speculative_b200.step import DecodeStep, layer_groups
 
     w = wl.WORKLOADS[name]
     if st is None:
@@ -633,7 +633,7 @@ def main():
 
     from datetime import timedelta
     from lossless_diffusion_speculative_b200.replicas import max_over_ranks, replica_throughput
-    from lossless_diffusion_speculative_b200.step import DecodeStep
+    from lossless_diffusion_speculative_b200.step import DecodeStep, layer_groups
 
     torch.cuda.set_device(local)
     if args.only:
@@ -726,13 +726,16 @@ def main():
             # waits only for what it reads.  A step's copies start once the
             # previous step is done with the buffers.
             cs = torch.cuda.Stream(device=dev)
-            chunk = 9
+            # layer groups: a one-layer first group (its copy is the only one
+            # not hidden behind compute), then groups of 8 and 9 layers
+            chunk = (1, 8, 9)
             egraphs = None if graphs is None else st.capture(stream, chunk=chunk)
             chunks, needs = [], {}
             if args.order == "cold":
                 for view, vn in ((0, "diff"), (1, "ar")):
-                    for c in range(0, st.L, chunk):
-                        sl = (view, slice(c, min(c + chunk, st.L)))
+                    for layers in layer_groups(st.L, chunk):
+                        c = layers.start
+                        sl = (view, slice(c, layers.stop))
                         needs[f"write_block_{vn}_{c}"] = needs[f"attn_{vn}_{c}"] = len(chunks)
                         chunks.append([("kb", sl), ("vb", sl), ("q", sl)])
             else:

@@ -31,6 +31,19 @@ from . import binding as ob
 from . import workloads as wl
 
 
+
+def layer_groups(L: int, chunk) -> list:
+    """Consecutive layer ranges covering [0, L): groups of ``chunk`` layers, or
+    of the sizes in ``chunk`` (a sequence; its last size repeats)."""
+    sizes = [int(chunk)] if isinstance(chunk, int) else [int(c) for c in chunk]
+    out, c, k = [], 0, 0
+    while c < L:
+        n = max(1, sizes[min(k, len(sizes) - 1)])
+        out.append(range(c, min(c + n, L)))
+        c += n
+        k += 1
+    return out
+
 @dataclass
 class StepResult:
     accepted: np.ndarray
@@ -147,10 +160,11 @@ class DecodeStep:
     def segments(self, chunk: int = 0, order: Optional[str] = None):
         """The step as ordered launch segments (timed separately by the bench).
 
-        With ``chunk`` > 0 (cold order) each view runs as layer groups of that
-        size, block install then attention per group: the same launches' work in
-        smaller segments, so that a caller feeding the step from the host can
-        start each group once its inputs have arrived.
+        With ``chunk`` (cold order: a group size, or a sequence of group sizes
+        repeated to cover the layers) each view runs as layer groups, block
+        install then attention per group: the same launches' work in smaller
+        segments, so that a caller feeding the step from the host can start
+        each group once its inputs have arrived.
         """
         order = self.order if order is None else order
         if order == "fused":
@@ -161,11 +175,11 @@ class DecodeStep:
         if order == "project_only":
             return [("project_diff", lambda: self._project_view(ob.DIFF)),
                     ("project_ar", lambda: self._project_view(ob.AR))]
-        if order == "cold" and chunk > 0:
+        if order == "cold" and chunk:
             segs = []
             for view, vn in ((ob.DIFF, "diff"), (ob.AR, "ar")):
-                for c in range(0, self.L, chunk):
-                    layers = range(c, min(c + chunk, self.L))
+                for layers in layer_groups(self.L, chunk):
+                    c = layers.start
                     segs.append((f"write_block_{vn}_{c}", lambda v=view, ls=layers: self._write_block(v, ls)))
                     segs.append((f"attn_{vn}_{c}", lambda v=view, ls=layers: [self._attn(v, l) for l in ls]))
             segs.append(("consensus_commit", self._tail))

@@ -14,11 +14,12 @@ from gpu_util import assert_attn_close
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("order,chunk", [("cold", 0), ("interleaved", 0), ("cold", 2)])
+@pytest.mark.parametrize("order,chunk", [("cold", 0), ("interleaved", 0), ("cold", 2), ("cold", (1, 2))])
 @pytest.mark.parametrize("graph", [False, True])
 def test_step_matches_oracle(order, chunk, graph):
-    # chunk > 0: each view as layer groups (install, then attention, per group),
-    # the segmentation the end-to-end benchmark feeds from the host
+    # chunk: each view as layer groups (install, then attention, per group),
+    # the segmentation the end-to-end benchmark feeds from the host (a group
+    # size, or group sizes with the last repeated)
     w = wl.WORKLOADS["qwen3_8b_step"].with_(ctx_lo=1500, ctx_hi=1500, layers=3,
                                             plant="fixed:9")
     st = DecodeStep(w, order=order)
