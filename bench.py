@@ -20,7 +20,9 @@ Multi-GPU runs are independent replicas (data parallel, no collective on the
 data path; "scaling": "weak").  The line also carries a ``configs`` block: the
 attention of both views, KV-read bandwidth and its fraction of the measured HBM
 bandwidth, and verified tokens/s for every workload of the decode step (medians
-of at least 50 L2-cold iterations each).
+of at least 50 L2-cold iterations each, with the fp64 oracle's time for the
+same step on the host cores), and the rows beyond the step: the fused LM head,
+the QKV projection, prefill and rejection verification.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead: each
 step runs whole layer-view attentions (every output row) of the same workload,
@@ -54,7 +56,7 @@ REF_BUDGET_S = 150.0                # reference arm: timed CPU seconds per run
 # DRAM traffic of one attn_tc_kernel launch on the headline workload, from the
 # ncu capture summarised in profiles/ (bytes read + written), keyed by the hash
 # of the kernel source it was taken on; reported as null once the source changes.
-NCU_TRAFFIC = {("qwen3_8b_step", "5fa3835a6b71460c"): 34.09e6}
+NCU_TRAFFIC = {("qwen3_8b_step", "5140e1e2a658290e"): 34.09e6}
 
 # The workloads of the configs block: (label, workload, order).  The 36-layer
 # step in its specified per-layer order (DIFF then AR per layer) is timed in
@@ -297,7 +299,7 @@ def config_of(w, args):
 
 
 # ----------------------------------------------------------------------------- configs block
-def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
+def measure_config(label, w, order, dev, stream, hbm, iters, st=None, oracle_timing=False):
     """Median µs of each launch segment of one workload's step over `iters`
     replays, L2 flushed before every attention segment (outside the events).
     `st` reuses an existing DecodeStep of the same workload."""
@@ -344,7 +346,34 @@ def measure_config(label, w, order, dev, stream, hbm, iters, st=None):
            "segments_us": med, "iters": iters,
            "timing": "median of per-segment CUDA events; L2 flushed before each attention segment"}
     del graphs, st
+    if oracle_timing:
+        out["oracle"] = oracle_step_time(w, tok, step_us)
     return out
+
+
+def oracle_step_time(w, tok, step_us):
+    """The fp64 oracle on the host cores for one step of workload w: one
+    layer-view attention (DIFF, every row) timed and scaled to the step's 2 x
+    layers views, plus one timed consensus.  The oracle's loops have no
+    data-dependent trip counts, so zero-filled inputs of the workload's shapes
+    and context lengths time exactly the work of seeded ones, without the
+    seconds of generating them (the arrays are written first, so no page is
+    first touched inside the timed region)."""
+    import oracle
+    q = np.full((w.B, w.K, w.Hq, w.D), 0.01, np.float32)
+    kc = np.full((w.B, w.Hkv, w.S_max, w.D), 0.01, np.float32)
+    ctx = np.asarray(w.ctx_lens(), np.int32)
+    logits = np.full((w.B, w.K, w.vocab), 0.5, np.float32)
+    prop = np.zeros((w.B, w.K), np.int32)
+    t0 = time.perf_counter()
+    oracle.attention(oracle.DIFF, q, kc, kc, ctx)
+    t1 = time.perf_counter()
+    oracle.consensus(logits, prop)
+    t2 = time.perf_counter()
+    ms = ((t1 - t0) * 2 * w.layers + (t2 - t1)) * 1e3
+    return {"ms_per_step": ms, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"one layer-view (all rows) x {2 * w.layers} views + one consensus",
+            "verified_tokens_per_s": tok / (ms * 1e-3), "gpu_step_speedup": ms * 1e3 / step_us}
 
 
 # ----------------------------------------------------------------------------- fused layer step
@@ -793,7 +822,8 @@ def main():
             for label, name, order in CONFIG_SET:
                 configs[label] = measure_config(label, wl.WORKLOADS[name], order, dev, stream,
                                                 hbm, CONFIG_ITERS,
-                                                st=st if name == w.name else None)
+                                                st=st if name == w.name else None,
+                                                oracle_timing=not args.no_cpu_baseline and name != w.name)
                 torch.cuda.empty_cache()
             configs["qwen3_8b_step_fused_qkv"] = measure_fused_step(
                 "qwen3_8b_step", dev, stream, hbm, CONFIG_ITERS // 2,
