@@ -755,14 +755,17 @@ def main():
             # waits only for what it reads.  A step's copies start once the
             # previous step is done with the buffers.
             cs = torch.cuda.Stream(device=dev)
-            # layer groups: a one-layer first group (its copy is the only one
-            # not hidden behind compute), then groups of 8 and 9 layers
-            chunk = (1, 8, 9)
+            # diffusion-view layer groups of 1, 2, 4, 8 and the rest: a layer's
+            # copies take about half its compute, so each group's inputs land
+            # while the groups before it run and only the first group's copy is
+            # exposed; the AR view's inputs arrive during the diffusion view,
+            # so it runs as one group
+            chunk = {"diff": (1, 2, 4, 8, 21), "ar": 64}
             egraphs = None if graphs is None else st.capture(stream, chunk=chunk)
             chunks, needs = [], {}
             if args.order == "cold":
                 for view, vn in ((0, "diff"), (1, "ar")):
-                    for layers in layer_groups(st.L, chunk):
+                    for layers in layer_groups(st.L, chunk[vn]):
                         c = layers.start
                         sl = (view, slice(c, layers.stop))
                         needs[f"write_block_{vn}_{c}"] = needs[f"attn_{vn}_{c}"] = len(chunks)

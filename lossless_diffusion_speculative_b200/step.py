@@ -161,7 +161,8 @@ class DecodeStep:
         """The step as ordered launch segments (timed separately by the bench).
 
         With ``chunk`` (cold order: a group size, or a sequence of group sizes
-        repeated to cover the layers) each view runs as layer groups, block
+        with the last repeated to cover the layers, or a dict of either per
+        view, keys "diff" and "ar") each view runs as layer groups, block
         install then attention per group: the same launches' work in smaller
         segments, so that a caller feeding the step from the host can start
         each group once its inputs have arrived.
@@ -178,7 +179,7 @@ class DecodeStep:
         if order == "cold" and chunk:
             segs = []
             for view, vn in ((ob.DIFF, "diff"), (ob.AR, "ar")):
-                for layers in layer_groups(self.L, chunk):
+                for layers in layer_groups(self.L, chunk[vn] if isinstance(chunk, dict) else chunk):
                     c = layers.start
                     segs.append((f"write_block_{vn}_{c}", lambda v=view, ls=layers: self._write_block(v, ls)))
                     segs.append((f"attn_{vn}_{c}", lambda v=view, ls=layers: [self._attn(v, l) for l in ls]))

@@ -14,7 +14,8 @@ from gpu_util import assert_attn_close
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("order,chunk", [("cold", 0), ("interleaved", 0), ("cold", 2), ("cold", (1, 2))])
+@pytest.mark.parametrize("order,chunk", [("cold", 0), ("interleaved", 0), ("cold", 2), ("cold", (1, 2)),
+                                         ("cold", {"diff": (1, 2), "ar": 3})])
 @pytest.mark.parametrize("graph", [False, True])
 def test_step_matches_oracle(order, chunk, graph):
     # chunk: each view as layer groups (install, then attention, per group),
