@@ -94,6 +94,7 @@ class DecodeStep:
         self.cons_ws = torch.empty(ob.orthrus_consensus_workspace_size(B, K, w.vocab),
                                    dtype=torch.uint8, device=dev)
         self.graphs = None
+        self.whole = None
         self.tc_path = ob.orthrus_attn_path(B, Hq, Hkv, D, K, dt) == 1
         self.project = False
         if project:
@@ -229,6 +230,22 @@ class DecodeStep:
         torch.cuda.synchronize()
         self.graphs = graphs
         return graphs
+
+    def capture_whole(self, stream: torch.cuda.Stream, order: Optional[str] = None) -> torch.cuda.CUDAGraph:
+        """One CUDA graph of the whole step: the reset and every segment."""
+        self.reset()
+        for _, fn in self.segments(0, order):      # warm: attributes set, plans cached
+            fn()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                self.reset()
+                for _, fn in self.segments(0, order):
+                    fn()
+        torch.cuda.synchronize()
+        self.whole = g
+        return g
 
     def result(self) -> StepResult:
         torch.cuda.synchronize()
