@@ -280,6 +280,20 @@ __global__ void __launch_bounds__(kVerifyThreads) rs_resid_kernel(RejectArgs p)
     const int b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     __shared__ ResidShared sh;
+    static_assert(ORTHRUS_MAX_BLOCK <= kVerifyThreads, "one block slot per thread");
+    // ---- thread i < K: slot i's proposal and its logits in both views, loaded
+    // before (and overlapping) the statistics merge
+    int x = -1;
+    float ar_x = 0.f, dr_x = 0.f, ua = 0.f;
+    if (threadIdx.x < p.K) {
+        const size_t row = (size_t)b * p.K + threadIdx.x;
+        x = p.proposed[row];
+        ua = p.u_accept[row];
+        if (x >= 0 && x < p.V) {
+            ar_x = p.ar[row * p.V + x];
+            dr_x = p.dr[row * p.V + x];
+        }
+    }
     // ---- each row's normalisers from its chunk statistics
     for (int i = warp; i < p.K; i += kVerifyThreads / 32) {
         const float4 *w = p.ws + ((size_t)b * p.K + i) * p.splits;
@@ -299,14 +313,13 @@ __global__ void __launch_bounds__(kVerifyThreads) rs_resid_kernel(RejectArgs p)
     if (threadIdx.x == 0) sh.first_rej = p.K;
     __syncthreads();
     // ---- every slot's accept decision; the first rejection wins
-    for (int i = threadIdx.x; i < p.K; i += kVerifyThreads) {
-        const size_t row = (size_t)b * p.K + i;
-        const int x = p.proposed[row];
+    if (threadIdx.x < p.K) {
+        const int i = threadIdx.x;
         bool keep = false;
         if (x >= 0 && x < p.V) {
-            const float px = fast_exp2(p.ar[row * p.V + x] * p.c - sh.rp[i].m) / sh.rp[i].l;
-            const float qx = fast_exp2(p.dr[row * p.V + x] * p.c - sh.rq[i].m) / sh.rq[i].l;
-            keep = p.u_accept[row] * qx < px;
+            const float px = fast_exp2(ar_x * p.c - sh.rp[i].m) / sh.rp[i].l;
+            const float qx = fast_exp2(dr_x * p.c - sh.rq[i].m) / sh.rq[i].l;
+            keep = ua * qx < px;
         }
         if (!keep) atomicMin(&sh.first_rej, i);
     }
