@@ -123,6 +123,7 @@ struct SkinnyShape {
     int BK;                              // token rows
     int Np;                              // token rows padded for the MMA's N
     int nst;                             // pipeline stages
+    int halves;                          // 128-row weight tiles per pass (1, or 2 without split-K)
     int32_t *status;
     // split-K (ksplit > 1): CTA u computes tile u / ksplit over hidden chunks
     // [k0(u % ksplit), k0(u % ksplit + 1)) into an fp32 partial; the last

@@ -77,7 +77,7 @@ __device__ __forceinline__ uint64_t column_max32(uint64_t (&k)[32], int lane)
 // [kMaxLmRows] int32, the last-CTA flag.
 constexpr uint32_t kExtraBytes = kMaxLmRows * 8 + kMaxLmRows * 4 + 16;
 
-template <int CPS>
+template <int CPS, bool PAIR>
 __global__ void __launch_bounds__(sg::kThreads, 1)
     lm_head_kernel(const __grid_constant__ sg::Maps mp, const LmHeadArgs p)
 {
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     pdl_wait();
     const int cid = blockIdx.x, grid = gridDim.x;
     if (warp < 4) {
-        sg::epilogue_tiles<false>(sm, sp, cid, grid, tmem, CPS,
+        sg::epilogue_tiles<false, PAIR>(sm, sp, cid, grid, tmem, CPS,
                            [&](int row, int, int, bool valid, int c0, const uint32_t (&x)[32]) {
                                uint64_t k[32];
 #pragma unroll
@@ -113,10 +113,10 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
                                if (c0 + lane < BK && m) atomicMax(ckeys + c0 + lane, (unsigned long long)m);
                            });
     } else if (warp == 4) {
-        if (lane == 0) sg::producer<CPS>(sm, sp, mp, cid, grid);
+        if (lane == 0) sg::producer<CPS, PAIR>(sm, sp, mp, cid, grid);
         __syncwarp();
     } else {
-        if (lane == 0) sg::mma_issuer<CPS>(sm, sp, cid, grid, tmem);
+        if (lane == 0) sg::mma_issuer<CPS, PAIR>(sm, sp, cid, grid, tmem);
         __syncwarp();
     }
     tc_fence_before();
@@ -173,13 +173,13 @@ bool lm_smem_ready(int dev)
     if (dev < 0 || dev >= kMaxDevices) return false;
     std::call_once(g_smem_once[dev], [dev] {
         const int lim = 226 * 1024;            // (room for the kernels' few bytes of static shared memory)
-        g_smem_ok[dev] =
-            cudaFuncSetAttribute(lmh::lm_head_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess &&
-            cudaFuncSetAttribute(lmh::lm_head_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess &&
-            cudaFuncSetAttribute(lmh::lm_head_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim) ==
-                cudaSuccess;
+        const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        g_smem_ok[dev] = cudaFuncSetAttribute(lmh::lm_head_kernel<1, false>, at, lim) == cudaSuccess &&
+                         cudaFuncSetAttribute(lmh::lm_head_kernel<2, false>, at, lim) == cudaSuccess &&
+                         cudaFuncSetAttribute(lmh::lm_head_kernel<4, false>, at, lim) == cudaSuccess &&
+                         cudaFuncSetAttribute(lmh::lm_head_kernel<1, true>, at, lim) == cudaSuccess &&
+                         cudaFuncSetAttribute(lmh::lm_head_kernel<2, true>, at, lim) == cudaSuccess &&
+                         cudaFuncSetAttribute(lmh::lm_head_kernel<4, true>, at, lim) == cudaSuccess;
         if (!g_smem_ok[dev]) cudaGetLastError();
     });
     return g_smem_ok[dev];
@@ -240,8 +240,12 @@ int orthrus_lm_head_consensus(const void *hidden, const void *lm_head, const int
     sp.ws_part = nullptr;
     sp.ws_count = nullptr;
     int cps = 1;
-    sg::pipeline_of(sp.Np, Hd / 64, &cps, &sp.nst);
-    const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, lmh::kExtraBytes);
+    // with 65-128 token rows every stage serves two 128-row weight tiles
+    // (the token rows, as many bytes as a weight tile, are then loaded once per
+    // two); fewer token rows keep four chunks per stage, more fill TMEM
+    sp.halves = sp.Np > 64 && sp.Np <= 128 ? 2 : 1;
+    sg::pipeline_of(sp.Np, Hd / 64, &cps, &sp.nst, sp.halves);
+    const sg::Layout L = sg::layout_of(sp.Np, sp.nst, cps, lmh::kExtraBytes, sp.halves);
 
     sg::Maps mp;
     if (!sg::encode_w(mp, 0, lm_head, V, Hd) || !sg::encode_x(mp, hidden, BK, Hd, sp.Np))
@@ -260,9 +264,15 @@ int orthrus_lm_head_consensus(const void *hidden, const void *lm_head, const int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cps == 4   ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<4>, mp, a)
-                          : cps == 2 ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<2>, mp, a)
-                                     : cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<1>, mp, a);
+    cudaError_t e;
+    if (sp.halves == 2)
+        e = cps == 4   ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<4, true>, mp, a)
+            : cps == 2 ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<2, true>, mp, a)
+                       : cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<1, true>, mp, a);
+    else
+        e = cps == 4   ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<4, false>, mp, a)
+            : cps == 2 ? cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<2, false>, mp, a)
+                       : cudaLaunchKernelEx(&cfg, lmh::lm_head_kernel<1, false>, mp, a);
     return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_LAUNCH;
 }
 

@@ -244,6 +244,7 @@ extern "C" int orthrus_qkv_project(const void *x, const void *w_q, const void *w
     sp.BK = B * K;
     sp.Np = qp.Np;
     sp.nst = qp.nst;
+    sp.halves = 1;
     sp.status = status;
     sp.ksplit = qp.ksplit;
     sp.ws_part = static_cast<float *>(workspace);

@@ -64,16 +64,17 @@ struct Maps {                            // one launch's tensor maps
     CUtensorMap x;                       // token rows: box (64, Np) or (64, Np / 2)
 };
 
-// Dynamic shared memory: [ring: stages x (CPS x A | CPS x X)] [barriers]
-// [tmem address, abort flag, 2 spare words] [the kernel's own region].
+// Dynamic shared memory: [ring: stages x (halves x CPS x A | CPS x X)]
+// [barriers] [tmem address, abort flag, 2 spare words] [the kernel's own
+// region].
 struct Layout {
     uint32_t stage_bytes, bars, misc, extra, total;
 };
 
-__host__ __device__ inline Layout layout_of(int Np, int nst, int cps, uint32_t extra_bytes)
+__host__ __device__ inline Layout layout_of(int Np, int nst, int cps, uint32_t extra_bytes, int halves = 1)
 {
     Layout l;
-    l.stage_bytes = (uint32_t)cps * (kABytes + (uint32_t)Np * 128u);
+    l.stage_bytes = (uint32_t)cps * ((uint32_t)halves * kABytes + (uint32_t)Np * 128u);
     l.bars = (uint32_t)nst * l.stage_bytes;
     l.misc = l.bars + B_COUNT * 8;
     l.extra = (l.misc + 16 + 15) & ~15u;
@@ -85,11 +86,15 @@ struct Smem {
     uint32_t base;
     uint8_t *ptr;
     Layout L;
-    int cps;
+    int cps, halves;
     volatile int *abort_flag;
     __device__ __forceinline__ uint32_t bar(int i) const { return base + L.bars + 8u * i; }
-    __device__ __forceinline__ uint32_t a_of(int st) const { return base + st * L.stage_bytes; }
-    __device__ __forceinline__ uint32_t b_of(int st) const { return a_of(st) + cps * kABytes; }
+    // weight chunks of half u of stage st (cps chunks of 16 KiB), then the token rows
+    __device__ __forceinline__ uint32_t a_of(int st, int u = 0) const
+    {
+        return base + st * L.stage_bytes + (uint32_t)(u * cps) * kABytes;
+    }
+    __device__ __forceinline__ uint32_t b_of(int st) const { return a_of(st) + (uint32_t)(halves * cps) * kABytes; }
     __device__ __forceinline__ uint8_t *extra() const { return ptr + L.extra; }
 };
 
@@ -101,11 +106,13 @@ __host__ __device__ __forceinline__ int split_k0(int s, int ksplit, int nk, int 
 }
 
 // The tiles of CTA `cid`'s range, in order; identical in every role.  Without
-// split-K the rows are cut into 16-row granules over the grid; with split-K
-// CTA cid owns 128-row tile cid / ksplit (tiles counted per segment) and the
-// hidden chunks [k_lo, k_hi) of split cid % ksplit.
+// split-K the rows are cut into 16-row granules over the grid and walked in
+// tiles of halves x 128 rows (two 128-row halves share each load of the
+// token rows when halves = 2); with split-K CTA cid owns 128-row tile
+// cid / ksplit (tiles counted per segment) and the hidden chunks [k_lo, k_hi)
+// of split cid % ksplit.
 struct TileIter {
-    int r0, hi;
+    int r0, hi, height;
     int e0, e1, e2;                      // segment ends (unused segments end at the last)
     int k_lo, k_hi;                      // hidden chunks of every tile
     __device__ __forceinline__ TileIter(const Shape &sh, int cid, int grid, int cps)
@@ -113,6 +120,7 @@ struct TileIter {
         e0 = sh.seg_end[0];
         e1 = sh.nseg > 1 ? sh.seg_end[1] : e0;
         e2 = sh.nseg > 2 ? sh.seg_end[2] : e1;
+        height = kTileRows * sh.halves;
         const int nk = sh.Hd / kChunk;
         if (sh.ksplit > 1) {
             int t = cid / sh.ksplit;
@@ -144,7 +152,7 @@ struct TileIter {
         seg_lo = seg == 0 ? 0 : seg == 1 ? e0 : e1;
         const int seg_hi = seg == 0 ? e0 : seg == 1 ? e1 : e2;
         a = r0;
-        b = r0 + kTileRows;
+        b = r0 + height;
         if (b > hi) b = hi;
         if (b > seg_hi) b = seg_hi;
         r0 = b;
@@ -152,7 +160,7 @@ struct TileIter {
     }
 };
 
-template <int CPS>
+template <int CPS, bool PAIR = false>
 __device__ __forceinline__ void producer(const Smem &sm, const Shape &sp, const Maps &mp, int cid, int grid)
 {
     const int nk = sp.Hd / kChunk;
@@ -165,8 +173,12 @@ __device__ __forceinline__ void producer(const Smem &sm, const Shape &sp, const 
     (void)nk;
     while (ok && ti.next(a, b, seg, seg_lo)) {
         const int nrows = b - a, y0 = a - seg_lo;
-        const int nb16 = (nrows + 15) >> 4;
-        const uint32_t a_bytes = nrows == kTileRows ? kABytes : (uint32_t)nb16 * 16u * 128u;
+        // rows of each 128-row weight half of the tile (the second may be short or empty)
+        const int n0 = nrows < kTileRows ? nrows : kTileRows, n1 = nrows - n0;
+        auto half_bytes = [](int n) -> uint32_t {
+            return n == kTileRows ? kABytes : (uint32_t)((n + 15) >> 4) * 16u * 128u;
+        };
+        const uint32_t a_bytes = half_bytes(n0) + (n1 > 0 ? half_bytes(n1) : 0u);
         for (int ks = ti.k_lo / CPS; ks < ti.k_hi / CPS; ++ks, ++it) {
             const int st = it % sp.nst;
             const uint32_t n = it / sp.nst;
@@ -180,12 +192,18 @@ __device__ __forceinline__ void producer(const Smem &sm, const Shape &sp, const 
 #pragma unroll
             for (int j = 0; j < CPS; ++j) {
                 const int kc = ks * CPS + j;
-                const uint32_t dst = sm.a_of(st) + j * kABytes;
-                if (nrows == kTileRows) {
-                    tma_load_2d_hint(dst, &mp.w[seg], full, kc * kChunk, y0, pol_w);
-                } else {
-                    for (int q = 0; q < nb16; ++q)
-                        tma_load_2d_hint(dst + q * 2048u, &mp.w16[seg], full, kc * kChunk, y0 + 16 * q, pol_w);
+#pragma unroll
+                for (int u = 0; u < (PAIR ? 2 : 1); ++u) {
+                    const int nu = u == 0 ? n0 : n1;
+                    if (nu <= 0) break;
+                    const uint32_t dst = sm.a_of(st, u) + j * kABytes;
+                    const int yu = y0 + kTileRows * u;
+                    if (nu == kTileRows) {
+                        tma_load_2d_hint(dst, &mp.w[seg], full, kc * kChunk, yu, pol_w);
+                    } else {
+                        for (int q = 0; q < ((nu + 15) >> 4); ++q)
+                            tma_load_2d_hint(dst + q * 2048u, &mp.w16[seg], full, kc * kChunk, yu + 16 * q, pol_w);
+                    }
                 }
                 const uint32_t xb = sm.b_of(st) + j * (uint32_t)sp.Np * 128u;
                 tma_load_2d_hint(xb, &mp.x, full, kc * kChunk, 0, pol_x);
@@ -201,11 +219,12 @@ __device__ __forceinline__ void producer(const Smem &sm, const Shape &sp, const 
     }
 }
 
-template <int CPS>
+template <int CPS, bool PAIR = false>
 __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int cid, int grid, uint32_t tmem)
 {
     const int nk = sp.Hd / kChunk;
-    const int nacc = 2 * sp.Np <= kTmemCols ? 2 : 1;
+    const int acc_cols = sp.halves * sp.Np;              // one accumulator: every half's Np columns
+    const int nacc = 2 * acc_cols <= kTmemCols ? 2 : 1;
     const bool split = sp.Np > 256;
     const int n_mma = split ? sp.Np / 2 : sp.Np;
     const uint32_t idesc = instr_desc(128, n_mma, false);
@@ -221,7 +240,8 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
             break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * sp.Np);
+        const bool second = PAIR && b - a > kTileRows;      // a second weight half in this tile
+        const uint32_t d = tmem + (uint32_t)(acc * acc_cols);
         const int ks0 = ti.k_lo / CPS;
         for (int ks = ks0; ks < ti.k_hi / CPS; ++ks, ++it) {
             const int st = it % sp.nst;
@@ -233,14 +253,19 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
 #pragma unroll
             for (int j = 0; j < CPS; ++j) {
                 const uint32_t xb = sm.b_of(st) + j * (uint32_t)sp.Np * 128u;
-                const uint64_t ad = smem_desc(sm.a_of(st) + j * kABytes, 16, 1024);
                 const uint64_t bd = smem_desc(xb, 16, 1024);
                 const uint64_t bd2 = smem_desc(xb + (uint32_t)n_mma * 128u, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {        // 16 hidden dims (32 bytes) per MMA
-                    const uint32_t on = ((ks - ks0) | j | kk) ? 1u : 0u;
-                    tc_mma_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, on);
-                    if (split) tc_mma_ss(d + (uint32_t)n_mma, ad + 2 * kk, bd2 + 2 * kk, idesc, on);
+                for (int u = 0; u < (PAIR ? 2 : 1); ++u) {  // (the token rows are shared by both halves)
+                    if (u == 1 && !second) break;
+                    const uint64_t ad = smem_desc(sm.a_of(st, u) + j * kABytes, 16, 1024);
+                    const uint32_t du = d + (uint32_t)(u * sp.Np);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {    // 16 hidden dims (32 bytes) per MMA
+                        const uint32_t on = ((ks - ks0) | j | kk) ? 1u : 0u;
+                        tc_mma_ss(du, ad + 2 * kk, bd + 2 * kk, idesc, on);
+                        if (split) tc_mma_ss(du + (uint32_t)n_mma, ad + 2 * kk, bd2 + 2 * kk, idesc, on);
+                    }
                 }
             }
             tc_commit(sm.bar(B_EMPTY + st));
@@ -260,12 +285,13 @@ __device__ __forceinline__ void mma_issuer(const Smem &sm, const Shape &sp, int 
 // With split-K each split writes its fp32 partial; the last split of the
 // tile to finish (per-tile counter, acquire/release) sums the partials in
 // split order and calls f with the sums.  named barrier 1 joins warps 0-3.
-template <bool SPLITK, class F>
+template <bool SPLITK, bool PAIR = false, class F>
 __device__ __forceinline__ bool epilogue_tiles(const Smem &sm, const Shape &sp, int cid, int grid, uint32_t tmem,
                                                int cps, F &&f)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nacc = 2 * sp.Np <= kTmemCols ? 2 : 1;
+    const int acc_cols = sp.halves * sp.Np;
+    const int nacc = 2 * acc_cols <= kTmemCols ? 2 : 1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const int rows = sp.seg_end[sp.nseg - 1];
     TileIter ti(sp, cid, grid, cps);
@@ -277,11 +303,17 @@ __device__ __forceinline__ bool epilogue_tiles(const Smem &sm, const Shape &sp, 
         const int row = a + warp * 32 + lane;
         const bool valid = row < b;
         if constexpr (!SPLITK) {
-            for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
-                uint32_t x[32];
-                tmem_ld32(lane_base + (uint32_t)(acc * sp.Np + c0), x);
-                tmem_wait_ld();
-                f(row, seg, seg_lo, valid, c0, x);
+            // every weight half of the tile: rows a + 128 u + (warp, lane), its Np columns
+#pragma unroll
+            for (int u = 0; u < (PAIR ? 2 : 1); ++u) {
+                if (u == 1 && b - a <= kTileRows) break;
+                const int row_u = row + u * kTileRows;
+                for (int c0 = 0; c0 < sp.Np && c0 < sp.BK; c0 += 32) {
+                    uint32_t x[32];
+                    tmem_ld32(lane_base + (uint32_t)(acc * acc_cols + u * sp.Np + c0), x);
+                    tmem_wait_ld();
+                    f(row_u, seg, seg_lo, row_u < b, c0, x);
+                }
             }
         } else {
             const int split = cid % sp.ksplit, tile = cid / sp.ksplit;
@@ -376,8 +408,9 @@ __device__ __forceinline__ uint32_t prologue(Smem &sm, uint8_t *smem_raw, const 
     const uint32_t aligned = (raw + 1023u) & ~1023u;
     sm.base = aligned;
     sm.ptr = smem_raw + (aligned - raw);
-    sm.L = layout_of(sp.Np, sp.nst, cps, extra_bytes);
+    sm.L = layout_of(sp.Np, sp.nst, cps, extra_bytes, sp.halves);
     sm.cps = cps;
+    sm.halves = sp.halves;
     sm.abort_flag = reinterpret_cast<volatile int *>(sm.ptr + sm.L.misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -426,17 +459,17 @@ __device__ __forceinline__ void tmem_free(uint32_t tmem)
 
 // Host: chunks per stage (the most of 4, 2, 1 that divide the hidden chunks
 // and leave two stages in the ring) and the stage count.
-inline void pipeline_of(int Np, int nk, int *cps, int *nst)
+inline void pipeline_of(int Np, int nk, int *cps, int *nst, int halves = 1)
 {
     *cps = 1;
     for (int c = 4; c >= 2; c >>= 1) {
-        const uint32_t sb = (uint32_t)c * (kABytes + (uint32_t)Np * 128u);
+        const uint32_t sb = (uint32_t)c * ((uint32_t)halves * kABytes + (uint32_t)Np * 128u);
         if (nk % c == 0 && 2 * sb <= kRingBudget) {
             *cps = c;
             break;
         }
     }
-    const uint32_t sb = (uint32_t)*cps * (kABytes + (uint32_t)Np * 128u);
+    const uint32_t sb = (uint32_t)*cps * ((uint32_t)halves * kABytes + (uint32_t)Np * 128u);
     const int n = (int)(kRingBudget / sb);
     *nst = n > kMaxStages ? kMaxStages : n;
 }

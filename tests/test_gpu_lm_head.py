@@ -49,6 +49,9 @@ SHAPES = {   # name: (B, K, Hd, V)
     "many_ctas_partial_tiles": (1, 32, 256, 20011),
     "two_mma_halves": (16, 32, 128, 3001),
     "rows_300": (10, 30, 64, 777),
+    "two_tile_passes_128_rows": (4, 32, 192, 40009),      # 270 vocabulary rows per CTA
+    "two_tile_passes_90_rows": (3, 30, 128, 30011),       # 203: a pair with a short second half
+    "two_tile_passes_vocab_under_a_pair": (2, 40, 64, 200),
 }
 
 
@@ -116,7 +119,7 @@ def test_lm_head_ties_lowest_index_and_workspace_reuse():
     assert (ram[0] == lo).all()
 
 
-@pytest.mark.parametrize("name", ["qwen3_8b_step", "qwen3_4b_ragged", "qwen3_1p7b_layer"])
+@pytest.mark.parametrize("name", ["qwen3_8b_step", "qwen3_4b_ragged", "qwen3_1p7b_layer", "qwen3_8b_long_k32"])
 def test_lm_head_full_size_planted(name):
     """Full Qwen3 vocabulary and width, in the benchmark's launch configuration:
     the planted argmax (margin ~7 against an fp32 bound < 0.4) is recovered
