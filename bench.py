@@ -792,7 +792,47 @@ def main():
             ready = [torch.cuda.Event() for _ in chunks]
             done = torch.cuda.Event()
 
+            # The whole end-to-end step as one CUDA graph: the copy stream
+            # forks from the step, each group's copies then an event, the
+            # step's segments each after its group's event, the result read
+            # back, the copy stream joined (one launch per step)
+            whole_e2e = None
+            if graphs is not None:
+                try:
+                    seg_fns = st.segments(chunk)
+                    fork, join = torch.cuda.Event(), torch.cuda.Event()
+                    for _, fn in seg_fns:
+                        fn()
+                    torch.cuda.synchronize()
+                    whole_e2e = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(whole_e2e, stream=stream):
+                        fork.record(stream)
+                        cs.wait_event(fork)
+                        with torch.cuda.stream(cs):
+                            for ev_i, ch in zip(ready, chunks):
+                                for n, v in ch:
+                                    d_t, h_t = (dst[n], host[n]) if v is None else (dst[n][v], host[n][v])
+                                    d_t.copy_(h_t, non_blocking=True)
+                                ev_i.record(cs)
+                            join.record(cs)
+                        st.reset()
+                        for name, fn in seg_fns:
+                            stream.wait_event(ready[needs[name]])
+                            fn()
+                        out_acc.copy_(st.accepted, non_blocking=True)
+                        out_nxt.copy_(st.next_token, non_blocking=True)
+                        stream.wait_event(join)
+                    torch.cuda.synchronize()
+                except Exception as exc:                  # (fall back to per-segment graphs)
+                    print(f"bench: whole-step end-to-end graph not captured ({exc}); "
+                          "per-segment graphs instead", file=sys.stderr)
+                    whole_e2e = None
+                    torch.cuda.synchronize()
+
             def e2e_step():
+                if whole_e2e is not None:
+                    whole_e2e.replay()
+                    return
                 if graphs is None:
                     for n in host:
                         dst[n].copy_(host[n], non_blocking=True)
@@ -830,7 +870,7 @@ def main():
             e2e_ms = a0.elapsed_time(a1)
             assert int(out_acc[0]) == int(res.accepted[0])
             e2e = (e2e_ms, e_steps, h2d, d2h)
-            egraphs = None
+            egraphs = whole_e2e = None
 
         # ---- every workload of the decode step, one at a time (rank 0 only)
         configs = None
