@@ -80,6 +80,58 @@ def test_host_checks_reject_bad_arguments_without_a_device(lib):
                                  None, None) == binding.ERR_ARG
 
 
+def test_host_checks_of_the_next_rows_without_a_device(lib):
+    """The fused LM head, rejection verification, QKV projection and prefill
+    reject bad arguments on the host, before any device call."""
+    vp = ctypes.c_void_p
+    ok = vp(16)
+    # LM head: NULL hidden; hidden size not a multiple of 64; more than 512 token rows;
+    # misaligned weight; workspace too small
+    assert lib.orthrus_lm_head_consensus(None, ok, ok, 1, 8, 100, 64, ok, ok, None, ok, 1 << 20,
+                                         None, None) == binding.ERR_ARG
+    assert lib.orthrus_lm_head_consensus(ok, ok, ok, 1, 8, 100, 100, ok, ok, None, ok, 1 << 20,
+                                         None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_lm_head_consensus(ok, ok, ok, 32, 32, 100, 64, ok, ok, None, ok, 1 << 20,
+                                         None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_lm_head_consensus(ok, vp(24), ok, 1, 8, 100, 64, ok, ok, None, ok, 1 << 20,
+                                         None, None) == binding.ERR_ALIGN
+    assert lib.orthrus_lm_head_consensus(ok, ok, ok, 1, 8, 100, 64, ok, ok, None, ok, 8,
+                                         None, None) == binding.ERR_WORKSPACE
+    assert lib.orthrus_lm_head_workspace_size(1, 32) >= 32 * 8 + 4
+    assert lib.orthrus_lm_head_workspace_size(0, 32) == 0 and lib.orthrus_lm_head_workspace_size(32, 32) == 0
+    # rejection: NULL draws; temperature <= 0; K above the block limit; misaligned logits
+    assert lib.orthrus_rejection_verify(ok, ok, ok, None, ok, 1.0, 1, 8, 100, ok, ok, ok, 1 << 20,
+                                        None, None) == binding.ERR_ARG
+    assert lib.orthrus_rejection_verify(ok, ok, ok, ok, ok, 0.0, 1, 8, 100, ok, ok, ok, 1 << 20,
+                                        None, None) == binding.ERR_ARG
+    assert lib.orthrus_rejection_verify(ok, ok, ok, ok, ok, 1.0, 1, 200, 100, ok, ok, ok, 1 << 20,
+                                        None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_rejection_verify(vp(20), ok, ok, ok, ok, 1.0, 1, 8, 100, ok, ok, ok, 1 << 20,
+                                        None, None) == binding.ERR_ALIGN
+    assert lib.orthrus_rejection_workspace_size(1, 200, 100) == 0
+    # QKV projection: NULL cache; hidden not a multiple of 64; D not a multiple of 16;
+    # Hq not a multiple of Hkv; misaligned x
+    assert lib.orthrus_qkv_project(ok, ok, ok, ok, ok, 1, 8, 256, 8, 2, 128, 64, ok, None, ok, ok,
+                                   1 << 20, None, None) == binding.ERR_ARG
+    assert lib.orthrus_qkv_project(ok, ok, ok, ok, ok, 1, 8, 250, 8, 2, 128, 64, ok, ok, ok, ok,
+                                   1 << 20, None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_qkv_project(ok, ok, ok, ok, ok, 1, 8, 256, 8, 2, 100, 64, ok, ok, ok, ok,
+                                   1 << 20, None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_qkv_project(ok, ok, ok, ok, ok, 1, 8, 256, 9, 2, 128, 64, ok, ok, ok, ok,
+                                   1 << 20, None, None) == binding.ERR_UNSUPPORTED
+    assert lib.orthrus_qkv_project(vp(18), ok, ok, ok, ok, 1, 8, 256, 8, 2, 128, 64, ok, ok, ok, ok,
+                                   1 << 20, None, None) == binding.ERR_ALIGN
+    assert lib.orthrus_qkv_workspace_size(1, 8, 250, 8, 2, 128) == 0
+    # prefill: NULL q; prompt longer than the cache; Hq not a multiple of Hkv
+    assert lib.orthrus_prefill_attn(0, None, ok, ok, 1, 64, 8, 2, 128, 128, 0.0, ok, ok, 1 << 20,
+                                    None, None) == binding.ERR_ARG
+    assert lib.orthrus_prefill_attn(0, ok, ok, ok, 1, 200, 8, 2, 128, 128, 0.0, ok, ok, 1 << 20,
+                                    None, None) == binding.ERR_ARG
+    assert lib.orthrus_prefill_attn(0, ok, ok, ok, 1, 64, 9, 2, 128, 128, 0.0, ok, ok, 1 << 20,
+                                    None, None) == binding.ERR_ARG
+    assert lib.orthrus_prefill_workspace_size(1, 64, 9, 2, 128, 0) == 0
+
+
 def test_device_status_is_a_per_call_word():
     """Every entry point that enqueues device work takes the caller's status
     word; the library keeps no global status (there is no get-status call),
@@ -88,7 +140,8 @@ def test_device_status_is_a_per_call_word():
     src = open(os.path.join(ROOT, "include", "orthrus.h")).read()
     decls = dict(re.findall(r"ORTHRUS_API\s+[\w\s\*]*?\b(orthrus_\w+)\s*\(([^;]*)\);", src))
     for name in ("orthrus_attn", "orthrus_attn_static", "orthrus_consensus",
-                 "orthrus_kv_commit", "orthrus_write_block"):
+                 "orthrus_kv_commit", "orthrus_write_block", "orthrus_lm_head_consensus",
+                 "orthrus_rejection_verify", "orthrus_qkv_project", "orthrus_prefill_attn"):
         assert re.search(r"int32_t\s*\*\s*status", decls[name]), name
         assert "hint" not in decls[name], name
     assert not any("status" in n for n in decls), sorted(decls)
